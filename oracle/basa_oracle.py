@@ -1,0 +1,337 @@
+"""CPU oracle for the BASA forward hot path (float64, numpy).
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it. The
+CUDA library never calls it, and it shares no code with the CUDA library.
+
+It states the operator the way the pages describe it, step by step, with no
+blocking, fusion or reordering beyond what the definition needs:
+
+  BASA = "Backend-Agnostic Sparse Attention for Fast High-Resolution Visual
+  Generation" (arXiv 2610.08772); sections below are that paper's.
+
+1. cyclic shift of the token grid (BASA §A.1: cyclic shift, reshape and
+   permutation form non-overlapping windows folded into the batch);
+2. non-overlapping windows of the shifted grid (BASA §3.1, §A.1);
+3. average-pooled global K/V over patches of the unshifted grid (BASA §3.2
+   "K/V-pooled global memory"; §A.1 "regular spatial reduction");
+4. content-adaptive routing: each query window adds the K/V of the windows whose
+   mean-pooled keys score highest against its mean-pooled query (BASA §3.3
+   "content-adaptive true-window routing");
+5. one softmax, scale 1/sqrt(d), over the concatenation own window | routed
+   windows | pooled tokens | text tokens (BASA §A.1: the local and text/global
+   branches are equivalent to one softmax over concatenated K/V);
+6. inverse shift of the output.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+  * shift convention Xr[t,y,x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W] (roll by -s);
+  * window ids are raster order over the window grid of the shifted frame;
+  * routing score = dot product of float64 window means of Q and K, the window
+    itself excluded, candidates = all other windows, ties to the lower id, the
+    chosen ids listed by descending score;
+  * text tokens are keys only (rows N.. of k and v); only visual queries are output;
+  * pooled tokens are listed in raster order of the pooled grid.
+
+Layouts: q, out [B, h, N, d]; k, v [B, h, N + n_text, d] (visual rows in raster
+(t, y, x) order, then text rows); kp, vp [B, h, Np, d]; route_idx [B, h, nWin, k].
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class Geometry:
+    """The arguments that fix the operator (besides the tensors themselves)."""
+
+    grid: tuple  # (T, H, W)
+    window: tuple  # (wt, wh, ww)
+    shift: tuple = (0, 0, 0)  # (st, sy, sx)
+    pool: tuple = (0, 0, 0)  # (pt, ph, pw); all zero = no pooled keys
+    n_text: int = 0
+    routed_k: int = 0
+
+    @property
+    def N(self):
+        T, H, W = self.grid
+        return T * H * W
+
+    @property
+    def win_grid(self):
+        return tuple(g // w for g, w in zip(self.grid, self.window))
+
+    @property
+    def n_win(self):
+        a, b, c = self.win_grid
+        return a * b * c
+
+    @property
+    def win_tokens(self):
+        a, b, c = self.window
+        return a * b * c
+
+    @property
+    def has_pool(self):
+        return all(p > 0 for p in self.pool)
+
+    @property
+    def n_pool(self):
+        if not self.has_pool:
+            return 0
+        return int(np.prod([g // p for g, p in zip(self.grid, self.pool)]))
+
+
+def to_grid(x, grid):
+    """[B, h, N, d] -> [B, h, T, H, W, d] (raster order t, y, x)."""
+    B, h, N, d = x.shape
+    return x.reshape(B, h, *grid, d)
+
+
+def cyclic_shift(X, shift):
+    """Xr[t, y, x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W]  (BASA §A.1 cyclic shift)."""
+    return np.roll(X, shift=tuple(-s for s in shift), axis=(2, 3, 4))
+
+
+def inverse_cyclic_shift(Xr, shift):
+    """Inverse of cyclic_shift: X[(t+st)%T, ...] = Xr[t, ...]."""
+    return np.roll(Xr, shift=tuple(shift), axis=(2, 3, 4))
+
+
+def window_partition(Xr, window):
+    """[B,h,T,H,W,d] -> [B,h,nWin,wt*wh*ww,d]; windows in raster order (BASA §A.1)."""
+    B, h, T, H, W, d = Xr.shape
+    wt, wh, ww = window
+    x = Xr.reshape(B, h, T // wt, wt, H // wh, wh, W // ww, ww, d)
+    x = x.transpose(0, 1, 2, 4, 6, 3, 5, 7, 8)
+    return x.reshape(B, h, (T // wt) * (H // wh) * (W // ww), wt * wh * ww, d)
+
+
+def window_unpartition(Xw, grid, window):
+    """Inverse of window_partition."""
+    B, h, nw, wtok, d = Xw.shape
+    T, H, W = grid
+    wt, wh, ww = window
+    x = Xw.reshape(B, h, T // wt, H // wh, W // ww, wt, wh, ww, d)
+    x = x.transpose(0, 1, 2, 5, 3, 6, 4, 7, 8)
+    return x.reshape(B, h, T, H, W, d)
+
+
+def pool_kv(k, v, geo: Geometry):
+    """Average of K and of V over each pt x ph x pw patch of the UNSHIFTED grid.
+
+    BASA §3.2 (K/V-pooled global memory: spatially pooled K/V gives every window a
+    cheap global context) and §A.1 (pooling is a regular spatial reduction). The
+    pooled tokens are in raster order of the pooled grid. Returns float64
+    [B, h, Np, d] twice.
+    """
+    T, H, W = geo.grid
+    pt, ph, pw = geo.pool
+    N = geo.N
+    res = []
+    for x in (k, v):
+        X = to_grid(np.asarray(x[:, :, :N], dtype=np.float64), geo.grid)
+        B, h, d = X.shape[0], X.shape[1], X.shape[-1]
+        P = X.reshape(B, h, T // pt, pt, H // ph, ph, W // pw, pw, d).mean(axis=(3, 5, 7))
+        res.append(P.reshape(B, h, -1, d))
+    return res[0], res[1]
+
+
+def window_means(q, k, geo: Geometry):
+    """Mean over each shifted window of Q and of K: float64 [B, h, nWin, d] each."""
+    N = geo.N
+    out = []
+    for x in (q, k):
+        X = to_grid(np.asarray(x[:, :, :N], dtype=np.float64), geo.grid)
+        Xw = window_partition(cyclic_shift(X, geo.shift), geo.window)
+        out.append(Xw.mean(axis=3))
+    return out[0], out[1]
+
+
+def route_windows(q, k, geo: Geometry):
+    """Top-k routed windows per query window (BASA §3.3, content-adaptive routing).
+
+    score[w, u] = mean(Q over window w) . mean(K over window u), u != w. The k
+    windows with the largest scores are kept, ties going to the lower window id,
+    listed by descending score. Returns (route_idx int32 [B,h,nWin,k],
+    scores float64 [B,h,nWin,nWin] with the diagonal set to -inf).
+    """
+    Qm, Km = window_means(q, k, geo)
+    S = np.einsum("bhwd,bhud->bhwu", Qm, Km)
+    nw = geo.n_win
+    S[..., np.arange(nw), np.arange(nw)] = -np.inf
+    B, h = S.shape[:2]
+    idx = np.zeros((B, h, nw, geo.routed_k), dtype=np.int32)
+    ids = np.arange(nw)
+    for b in range(B):
+        for hh in range(h):
+            for w in range(nw):
+                cand = ids[ids != w]
+                sc = S[b, hh, w, cand]
+                order = np.lexsort((cand, -sc))  # primary: score descending, then id ascending
+                idx[b, hh, w] = cand[order[: geo.routed_k]]
+    return idx, S
+
+
+def round_to_bf16(x):
+    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64.
+
+    Used to hand the oracle's pooled K/V to a bfloat16 kernel; done through float32
+    (exact for the float32 path) with the bit arithmetic written out.
+    """
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def basa_attention(q, k, v, geo: Geometry, kp=None, vp=None, route_idx=None, return_keys=False):
+    """BASA forward: out [B, h, N, d] float64.
+
+    For each query i of shifted window w: out_i = softmax_j(q_i . k_j / sqrt(d)) v_j
+    over the keys [own window | routed windows (route order) | pooled | text]
+    (BASA §3.1-§3.3, §A.1), then the output is shifted back to the original grid.
+    ``kp``/``vp`` default to pool_kv(); ``route_idx`` defaults to route_windows().
+    """
+    q64 = np.asarray(q, dtype=np.float64)
+    k64 = np.asarray(k, dtype=np.float64)
+    v64 = np.asarray(v, dtype=np.float64)
+    B, h, N, d = q64.shape
+    assert N == geo.N
+    if geo.has_pool and kp is None:
+        kp, vp = pool_kv(k64, v64, geo)
+    if geo.routed_k > 0 and route_idx is None:
+        route_idx, _ = route_windows(q64, k64, geo)
+
+    def windows(x):
+        return window_partition(cyclic_shift(to_grid(x[:, :, :N], geo.grid), geo.shift), geo.window)
+
+    Qw, Kw, Vw = windows(q64), windows(k64), windows(v64)
+    Ow = np.empty_like(Qw)
+    scale = 1.0 / np.sqrt(d)
+    for b in range(B):
+        for hh in range(h):
+            for w in range(geo.n_win):
+                kparts, vparts = [Kw[b, hh, w]], [Vw[b, hh, w]]
+                for r in range(geo.routed_k):
+                    u = int(route_idx[b, hh, w, r])
+                    kparts.append(Kw[b, hh, u])
+                    vparts.append(Vw[b, hh, u])
+                if geo.has_pool:
+                    kparts.append(np.asarray(kp[b, hh], dtype=np.float64))
+                    vparts.append(np.asarray(vp[b, hh], dtype=np.float64))
+                if geo.n_text > 0:
+                    kparts.append(k64[b, hh, N:])
+                    vparts.append(v64[b, hh, N:])
+                Kc = np.concatenate(kparts, axis=0)
+                Vc = np.concatenate(vparts, axis=0)
+                s = (Qw[b, hh, w] @ Kc.T) * scale
+                s = s - s.max(axis=1, keepdims=True)
+                p = np.exp(s)
+                p = p / p.sum(axis=1, keepdims=True)
+                Ow[b, hh, w] = p @ Vc
+    O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)
+    return O.reshape(B, h, N, d)
+
+
+def window_of_token(geo: Geometry):
+    """Window id of every token of the ORIGINAL grid, computed without any roll.
+
+    A token at original coordinate c (per axis) sits at shifted coordinate
+    (c - s) mod G, hence in window ((c - s) mod G) // w along that axis.
+    """
+    T, H, W = geo.grid
+    wt, wh, ww = geo.window
+    st, sy, sx = geo.shift
+    nWt, nWy, nWx = geo.win_grid
+    t = ((np.arange(T) - st) % T) // wt
+    y = ((np.arange(H) - sy) % H) // wh
+    x = ((np.arange(W) - sx) % W) // ww
+    return ((t[:, None, None] * nWy + y[None, :, None]) * nWx + x[None, None, :]).reshape(-1)
+
+
+def dense_masked_attention(q, k, v, geo: Geometry, route_idx=None, kp=None, vp=None):
+    """Independent formulation: dense attention in the original frame with a key mask.
+
+    Keys are [all N visual tokens | pooled | text]; query i may see visual key j
+    iff win(j) == win(i) or win(j) is one of win(i)'s routed windows; pooled and
+    text keys are always visible. No roll, no window gather.
+    """
+    q64 = np.asarray(q, dtype=np.float64)
+    k64 = np.asarray(k, dtype=np.float64)
+    v64 = np.asarray(v, dtype=np.float64)
+    B, h, N, d = q64.shape
+    win = window_of_token(geo)
+    if geo.has_pool and kp is None:
+        kp, vp = pool_kv(k64, v64, geo)
+    out = np.empty_like(q64)
+    for b in range(B):
+        for hh in range(h):
+            allowed = win[:, None] == win[None, :]
+            if geo.routed_k > 0:
+                routed = np.zeros((geo.n_win, geo.n_win), dtype=bool)
+                for w in range(geo.n_win):
+                    routed[w, route_idx[b, hh, w]] = True
+                allowed = allowed | routed[win[:, None], win[None, :]]
+            keys = [k64[b, hh, :N]]
+            vals = [v64[b, hh, :N]]
+            extra = 0
+            if geo.has_pool:
+                keys.append(np.asarray(kp[b, hh], dtype=np.float64))
+                vals.append(np.asarray(vp[b, hh], dtype=np.float64))
+                extra += kp.shape[2]
+            if geo.n_text > 0:
+                keys.append(k64[b, hh, N:])
+                vals.append(v64[b, hh, N:])
+                extra += geo.n_text
+            mask = np.concatenate([allowed, np.ones((N, extra), dtype=bool)], axis=1)
+            Kc = np.concatenate(keys, axis=0)
+            Vc = np.concatenate(vals, axis=0)
+            s = (q64[b, hh] @ Kc.T) / np.sqrt(d)
+            s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=1, keepdims=True)
+            out[b, hh] = p @ Vc
+    return out
+
+
+def attention_rows(q, k, v, geo: Geometry, b, hh, tokens, kp=None, vp=None, route_idx=None):
+    """Output rows for a sample of ORIGINAL token indices of one (b, head), float64.
+
+    Used to check large problems on a sample; it applies the same definition as
+    basa_attention to just the listed queries, finding each query's window by
+    window_of_token().
+    """
+    N = geo.N
+    d = q.shape[-1]
+    win = window_of_token(geo)
+    k64 = np.asarray(k[b, hh], dtype=np.float64)
+    v64 = np.asarray(v[b, hh], dtype=np.float64)
+    q64 = np.asarray(q[b, hh], dtype=np.float64)
+    members = {}
+    res = np.empty((len(tokens), d))
+    for n, i in enumerate(tokens):
+        w = int(win[i])
+        wins = [w] + ([int(u) for u in route_idx[b, hh, w]] if geo.routed_k > 0 else [])
+        rows = []
+        for u in wins:
+            if u not in members:
+                members[u] = np.nonzero(win == u)[0]
+            rows.append(members[u])
+        kparts = [k64[np.concatenate(rows)]]
+        vparts = [v64[np.concatenate(rows)]]
+        if geo.has_pool:
+            kparts.append(np.asarray(kp[b, hh], dtype=np.float64))
+            vparts.append(np.asarray(vp[b, hh], dtype=np.float64))
+        if geo.n_text > 0:
+            kparts.append(k64[N:])
+            vparts.append(v64[N:])
+        Kc = np.concatenate(kparts)
+        Vc = np.concatenate(vparts)
+        s = (Kc @ q64[i]) / np.sqrt(d)
+        p = np.exp(s - s.max())
+        res[n] = (p / p.sum()) @ Vc
+    return res

@@ -1,0 +1,65 @@
+"""Planted mistakes in a copy of the oracle must be caught by the pins.
+
+Each case edits the oracle's source text (a wrong sign, a dropped term, a wrong
+axis, a transposed order), builds a throw-away module from it, points the pin
+tests at that module and expects at least one of them to fail. The real oracle
+is never modified.
+"""
+import inspect
+import sys
+import types
+
+import pytest
+
+from oracle import basa_oracle
+from tests import test_oracle as pins
+
+MUTATIONS = [
+    # (name, old text, new text, pins that must catch it)
+    ("shift sign", "np.roll(X, shift=tuple(-s for s in shift)", "np.roll(X, shift=tuple(s for s in shift)", ["shift_membership"]),
+    ("window order", "x.transpose(0, 1, 2, 4, 6, 3, 5, 7, 8)", "x.transpose(0, 1, 6, 4, 2, 3, 5, 7, 8)", ["shift_membership"]),
+    ("mask sign", "t = ((np.arange(T) - st) % T) // wt", "t = ((np.arange(T) + st) % T) // wt", ["shift_membership"]),
+    ("pool patch stride", "X.reshape(B, h, T // pt, pt, H // ph, ph, W // pw, pw, d)", "X.reshape(B, h, pt, T // pt, ph, H // ph, pw, W // pw, d)", ["pool_centre"]),
+    ("route order", "np.lexsort((cand, -sc))", "np.lexsort((cand, sc))", ["route_planted", "route_brute"]),
+    ("route self", ["S[..., np.arange(nw), np.arange(nw)] = -np.inf", "cand = ids[ids != w]"], ["pass", "cand = ids"], ["route_planted", "route_brute"]),
+    ("route tie", "np.lexsort((cand, -sc))", "np.lexsort((-cand, -sc))", ["route_ties"]),
+    ("drop text keys", "                    kparts.append(k64[b, hh, N:])\n                    vparts.append(v64[b, hh, N:])\n                Kc", "                    pass\n                Kc", ["dense_masked", "constant_scores"]),
+    ("drop pooled keys", "                    kparts.append(np.asarray(kp[b, hh], dtype=np.float64))\n                    vparts.append(np.asarray(vp[b, hh], dtype=np.float64))\n                if geo.n_text > 0:\n                    kparts.append(k64[b, hh, N:])", "                    pass\n                if geo.n_text > 0:\n                    kparts.append(k64[b, hh, N:])", ["dense_masked"]),
+    ("scale", "scale = 1.0 / np.sqrt(d)", "scale = 1.0 / d", ["closed_form"]),
+    ("softmax axis", "s = s - s.max(axis=1, keepdims=True)\n                p = np.exp(s)\n                p = p / p.sum(axis=1, keepdims=True)\n                Ow", "s = s - s.max(axis=0, keepdims=True)\n                p = np.exp(s)\n                p = p / p.sum(axis=0, keepdims=True)\n                Ow", ["closed_form", "rows_sum"]),
+    ("routed window id", "u = int(route_idx[b, hh, w, r])", "u = int(route_idx[b, hh, (w + 1) % geo.n_win, r])", ["dense_masked"]),
+    ("unshift output", "O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)", "O = window_unpartition(Ow, geo.grid, geo.window)", ["dense_masked"]),
+]
+
+PINS = {
+    "shift_membership": lambda: pins.test_shift_membership_golden(),
+    "pool_centre": lambda: pins.test_pool_of_token_index_is_patch_centre(),
+    "route_planted": lambda: pins.test_route_planted_winner_and_self_excluded(),
+    "route_brute": lambda: [pins.test_route_matches_brute_force(g) for g in (pins.O.Geometry(grid=(1, 8, 12), window=(1, 4, 3), shift=(0, 1, 2), routed_k=3),)],
+    "route_ties": lambda: pins.test_route_ties_go_to_lower_id(),
+    "dense_masked": lambda: [pins.test_attention_matches_dense_masked_brute_force(g) for g in pins.TINY_GEOS],
+    "constant_scores": lambda: [pins.test_constant_scores_give_mean_of_key_values(g) for g in pins.TINY_GEOS],
+    "closed_form": lambda: pins.test_closed_form_whole_grid_is_dense_sdpa(),
+    "rows_sum": lambda: [pins.test_softmax_rows_sum_to_one(g) for g in pins.TINY_GEOS],
+}
+
+
+def _mutant(monkeypatch, old, new):
+    src = inspect.getsource(basa_oracle)
+    olds, news = (old, new) if isinstance(old, list) else ([old], [new])
+    for o, n in zip(olds, news):
+        assert src.count(o) >= 1, o
+        src = src.replace(o, n, 1)
+    mod = types.ModuleType("oracle_mutant")
+    monkeypatch.setitem(sys.modules, "oracle_mutant", mod)
+    exec(compile(src, "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new,catchers", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(monkeypatch, name, old, new, catchers):
+    mutant = _mutant(monkeypatch, old, new)
+    monkeypatch.setattr(pins, "O", mutant)
+    for pin in catchers:
+        with pytest.raises(Exception):
+            PINS[pin]()
