@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the BASA forward hot path (one layer = pool [+ route] + attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload flux2k] [--impl ours|reference]
+
+A step is one layer call over one batch of synthetic inputs already resident in
+HBM; consecutive steps walk the workload's shift cycle (one shift per layer).
+Rank 0 prints ONE JSON line. Multi-GPU runs (torchrun) give every rank its own
+copy of the workload (the path shards over (batch, head) with no exchange),
+time on the device and report the max over ranks ("scaling": "weak").
+
+The reference arm (--impl reference) times the float64 CPU oracle on the host
+cores on a bounded sample of the same workload (the oracle is the only other
+implementation there is).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_window_attention_b200 import accounting, synth  # noqa: E402
+
+METRIC = "shifted-window attn fwd effective TFLOP/s & % of B200 BF16 peak; ms/layer"
+ATTN_SOURCE = os.path.join(ROOT, "sparse_window_attention_b200", "csrc", "attn_bf16_sm100.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (sha256 recorded in the summary); else None."""
+    prof = os.path.join(ROOT, "profiles", f"attn_bf16_{workload}.md")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    sha = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != sha:
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- our arm
+
+
+def run_ours(args, world, rank, local):
+    from sparse_window_attention_b200.layer import BasaLayer
+
+    wl = synth.WORKLOADS[args.workload]
+    cnt = accounting.workload_counts(wl)
+    shifts = synth.SHIFT_CYCLES[args.workload]
+    q, k, v = synth.make_inputs(wl, seed=args.seed + rank)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        sh = shifts[i % len(shifts)]
+        if layer.has_pool:
+            layer.pool_kv(kd, vd, sh)
+        if layer.routed_k > 0:
+            layer.route(qd, kd, sh)
+        if ev is not None:
+            ev[0].record(stream)
+        layer.attention(qd, kd, vd, out, sh)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+
+    # timed region: K whole steps
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = t0.elapsed_time(t1) / args.steps
+    step_ms = max_over_ranks(step_ms, world)
+    assert layer.device_error() == 0
+
+    # attention-kernel duration (events bracketing each attention launch)
+    n_ev = min(args.steps, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    for i in range(n_ev):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    flops = cnt["attn_flops"]
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = kernel_traffic(ATTN_SOURCE, args.workload)
+    clocks = sampler.summary()
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} grid={'x'.join(map(str, wl.grid))} "
+                        f"window={'x'.join(map(str, wl.window))} shifts={shifts} pool={'x'.join(map(str, wl.pool))} "
+                        f"text={wl.n_text} routed_k={wl.routed_k}",
+            "keys_per_query": cnt["keys_per_query"],
+            "attn_gflop_per_layer": round(flops / 1e9, 2),
+            "parallelism": f"replica per GPU x{world}",
+            "l2": f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush",
+        },
+        "pct_of_peak": {
+            "step_vs_measured_burst": round(value / world / peak, 4),
+            "step_vs_nominal_2250": round(value / world / 2250.0, 4),
+        },
+        "roofline": {
+            "kernel": "attn_bf16_kernel",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 1.59 PF/s",
+            "traffic": traffic,
+            "attn_ms": round(attn_ms, 4),
+        },
+        "clocks": clocks,
+        "gpu_launches": args.steps * layer.launches_per_forward(),
+    }
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world)
+    if not args.no_extra and world == 1 and args.workload != "wan":
+        res["also_wan"] = run_also(args, "wan")
+    return res
+
+
+def run_e2e(args, layer, q, k, v, shifts, flops, world):
+    """Same metric through the public API with host (pinned) buffers: every step
+    copies q, k, v host->device, runs the layer and copies the output back."""
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    hout = torch.empty_like(hq).pin_memory()
+    dq, dk, dv = torch.empty_like(hq, device="cuda"), torch.empty_like(hk, device="cuda"), torch.empty_like(hv, device="cuda")
+    dout = torch.empty_like(dq)
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, args.e2e_steps))
+
+    def step(i):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        layer.forward(dq, dk, dv, shifts[i % len(shifts)], out=dout)
+        hout.copy_(dout, non_blocking=True)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    esz = hq.element_size()
+    return {
+        "value": round(world * flops / (ms * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(ms, 3),
+        "steps": steps,
+        "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * esz,
+        "d2h_bytes_per_step": hout.numel() * esz,
+    }
+
+
+def run_also(args, name):
+    """Secondary workload on the same GPU (context for the headline line)."""
+    sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True,
+                                "steps": max(50, args.steps // 4)})
+    r = run_ours(sub, 1, 0, int(os.environ.get("LOCAL_RANK", "0")))
+    return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "gpu_launches")}
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+
+
+def cpu_oracle_sample(wl, budget_s: float, max_units: int | None = None):
+    """Time the float64 oracle on (head, window) units of the workload: pooling of
+    the head plus attention of one window's queries; returns (TFLOP/s, units, seconds, threads)."""
+    from oracle import basa_oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    geo = O.Geometry(grid=wl.grid, window=wl.window, shift=wl.shift, pool=wl.pool, n_text=wl.n_text, routed_k=wl.routed_k)
+    q, k, v = synth.make_inputs(wl, seed=0, heads=[0])
+    q64, k64, v64 = (t.to(torch.float32).numpy().astype(np.float64) for t in (q, k, v))
+    cnt = accounting.workload_counts(wl)
+    flops_per_unit = cnt["attn_flops"] / (wl.B * wl.heads * cnt["n_win"])
+    win = O.window_of_token(geo)
+    units, t0 = 0, time.perf_counter()
+    route = O.route_windows(q64, k64, geo)[0] if geo.routed_k else None
+    kp, vp = O.pool_kv(k64, v64, geo) if geo.has_pool else (None, None)
+    while True:
+        w = units % cnt["n_win"]
+        if w == 0 and units > 0 and geo.has_pool:
+            kp, vp = O.pool_kv(k64, v64, geo)
+        toks = np.nonzero(win == w)[0]
+        O.attention_rows(q64, k64, v64, geo, 0, 0, toks, kp=kp, vp=vp, route_idx=route)
+        units += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_units and units >= max_units):
+            break
+    return units * flops_per_unit / el / 1e12, units, el, threads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[args.workload]
+    cnt = accounting.workload_counts(wl)
+    per_step_budget = min(0.5, 150.0 / max(1, args.steps + args.warmup))
+    cpu_oracle_sample(wl, 0.0, max_units=max(1, args.warmup))
+    tflops, units, el, threads = cpu_oracle_sample(wl, per_step_budget * args.steps)
+    step_ms = el / max(1, args.steps) * 1e3
+    sample = f"{units} (head, window) units of {args.workload} (head 0): oracle pooling + all queries of a window, float64 numpy"
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(tflops, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "keys_per_query": cnt["keys_per_query"]},
+        "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(tflops, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="flux2k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workload")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    res = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tflops, units, el, threads = cpu_oracle_sample(synth.WORKLOADS[args.workload], args.cpu_budget)
+        res["cpu_baseline"] = {
+            "value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{units} (head, window) units of {args.workload}, head 0, {el:.1f} s, float64 numpy",
+        }
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

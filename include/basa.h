@@ -1,0 +1,163 @@
+/*
+ * basa.h — C ABI of the BASA forward hot path on NVIDIA B200 (sm_100a).
+ *
+ * BASA = "Backend-Agnostic Sparse Attention for Fast High-Resolution Visual
+ * Generation" (arXiv 2610.08772). One layer of BASA replaces visual
+ * self-attention by attention over shifted non-overlapping windows whose key
+ * set is extended with pooled global K/V, optional routed windows and text
+ * tokens. Three calls make one layer:
+ *
+ *   basa_pool_kv          pooled global K/V            (BASA §3.2, §A.1)
+ *   basa_route_windows    top-k routed windows          (BASA §3.3, §A.2)
+ *   basa_window_attn_fwd  shifted-window attention      (BASA §3.1, §A.1)
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ * Pointers. Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *   library never allocates, frees, copies to the host or synchronises. Tensor
+ *   pointers must be 16-byte aligned (route_idx / route_score: 4-byte).
+ * Layouts (row-major, innermost last; N = T*H*W visual tokens in raster order
+ *   t, y, x; Np = (T/pt)*(H/ph)*(W/pw) pooled tokens in raster order of the
+ *   pooled grid; nWin = (T/wt)*(H/wh)*(W/ww)):
+ *     q, out        [B, heads, N, head_dim]
+ *     k, v          [B, heads, N + n_text, head_dim]   visual rows, then text rows
+ *     kp, vp        [B, heads, Np, head_dim]
+ *     route_idx     int32 [B, heads, nWin, routed_k]
+ *     route_score   float [B, heads, nWin, routed_k]
+ *   Element type: bfloat16 (BASA_BF16) or float32 (BASA_F32) for q, k, v, kp,
+ *   vp and out alike.
+ * Cyclic shift. The shifted grid is Xr[t,y,x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W];
+ *   windows are the non-overlapping wt x wh x ww blocks of Xr, numbered in
+ *   raster order of the window grid. Outputs are written at the ORIGINAL (not
+ *   shifted) positions.
+ * Streams. All work is enqueued on `stream` (0 = legacy default stream); each
+ *   call returns as soon as its kernels are launched. Calls on one stream are
+ *   ordered by the stream.
+ * Errors. Arguments are checked on the host before anything is launched; an
+ *   invalid call returns an error code and launches nothing. A launch failure
+ *   returns BASA_ERR_CUDA. No entry point aborts, traps or prints.
+ * Threads. Entry points are reentrant; the only library state is the lazily
+ *   resolved driver entry point used to encode TMA tensor maps.
+ */
+#ifndef BASA_H
+#define BASA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *basa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  BASA_OK = 0,
+  BASA_ERR_INVALID_ARG = 1,    /* null pointer, bad enum, negative count, misaligned pointer */
+  BASA_ERR_SHAPE = 2,          /* window or pool patch does not divide the grid, shift out of range */
+  BASA_ERR_UNSUPPORTED = 3,    /* valid but not built: e.g. bfloat16 attention with head_dim 64 */
+  BASA_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  BASA_ERR_DEVICE_TIMEOUT = 5  /* a bounded wait inside a kernel expired (reported via dev_err) */
+} basa_status;
+
+typedef enum { BASA_BF16 = 0, BASA_F32 = 1 } basa_dtype;
+
+/* Device error word bits written (atomicOr) into *dev_err by the kernels. */
+#define BASA_DEVERR_TIMEOUT_PRODUCER 0x1
+#define BASA_DEVERR_TIMEOUT_MMA 0x2
+#define BASA_DEVERR_TIMEOUT_SOFTMAX 0x4
+
+/* Test hook for basa_params.flags: the attention kernel's loader skips the TMA
+ * load of the first key tile, so every wait on it runs into its time limit and
+ * the kernel returns with BASA_DEVERR_TIMEOUT_* set. Never set in normal use. */
+#define BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD 0x1u
+
+typedef struct {
+  int B, heads, head_dim;  /* head_dim in {64, 128}                                    */
+  int T, H, W;             /* token grid; T = 1 for images                             */
+  int wt, wh, ww;          /* window extents; each divides T, H, W                     */
+  int st, sy, sx;          /* per-layer cyclic shift; 0 <= s < grid extent             */
+  int pt, ph, pw;          /* pool patch; all 0 = no pooled keys; else each divides    */
+  int n_text;              /* text rows appended after the N visual rows of k and v   */
+  int routed_k;            /* 0 = no routing; else 1 <= routed_k <= min(16, nWin - 1)  */
+  basa_dtype dtype;
+  int32_t *dev_err;        /* nullable DEVICE word; kernels OR BASA_DEVERR_* bits into it
+                              when a bounded wait expires. Read it after the stream has
+                              synchronised; map it with basa_device_error_status().    */
+  uint32_t flags;          /* 0, or BASA_FLAG_TEST_* hooks                              */
+  uint32_t wait_timeout_us;/* limit of each bounded wait inside the attention kernel;
+                              0 = default (2,000,000 us)                               */
+} basa_params;
+
+/*
+ * basa_pool_kv — pooled global K/V (BASA §3.2 "K/V-pooled global memory";
+ * §A.1: pooling is a regular spatial reduction of the UNSHIFTED grid).
+ *
+ *   kp[b,h,P,:] = mean of k[b,h,n,:] over the tokens n of patch P
+ *   vp[b,h,P,:] = mean of v[b,h,n,:] over the same tokens
+ * where patch P is the P-th pt x ph x pw block of the unshifted token grid in
+ * raster order. Text rows are not pooled. Sums are accumulated in float32 and
+ * the mean is rounded once to the element type (round to nearest even).
+ * Requires pt, ph, pw > 0. Reads k, v; writes kp, vp (no aliasing allowed).
+ */
+basa_status basa_pool_kv(const void *k, const void *v, void *kp, void *vp,
+                         const basa_params *p, basa_stream_t stream);
+
+/*
+ * basa_route_workspace_bytes — size of the caller-allocated device workspace
+ * basa_route_windows needs (the float32 window means of Q and K:
+ * 2 * B * heads * nWin * head_dim * 4 bytes). Returns 0 for invalid params.
+ */
+size_t basa_route_workspace_bytes(const basa_params *p);
+
+/*
+ * basa_route_windows — content-adaptive true-window routing (BASA §3.3; §A.2:
+ * routed windows are added as uncompressed K/V to each query window).
+ *
+ *   Qm[w] = mean of q over the tokens of shifted window w     (float32)
+ *   Km[u] = mean of k over the tokens of shifted window u     (float32)
+ *   score[w,u] = Qm[w] . Km[u]  for u != w
+ *   route_idx[b,h,w,:] = the routed_k windows u with the largest scores,
+ *                        ties to the lower id, by descending score
+ *   route_score[b,h,w,:] = their scores (optional: pass NULL to skip)
+ * Requires routed_k >= 1. `workspace` is a device buffer of at least
+ * basa_route_workspace_bytes(p) bytes, 16-byte aligned; its contents on entry
+ * are ignored and on return are the window means [2][B][heads][nWin][head_dim].
+ */
+basa_status basa_route_windows(const void *q, const void *k, int32_t *route_idx,
+                               float *route_score, void *workspace,
+                               const basa_params *p, basa_stream_t stream);
+
+/*
+ * basa_window_attn_fwd — shifted-window attention forward (BASA §3.1 shifted
+ * windows; §A.1: the local and global/text branches equal ONE softmax over the
+ * concatenated K/V, which is what is computed here in a single pass).
+ *
+ * For every query token i of shifted window w:
+ *   keys(i) = tokens of w | tokens of route_idx[b,h,w,0..routed_k-1]
+ *             | the Np pooled tokens (kp, vp) | the n_text text rows of k, v
+ *   out[i]  = sum_j softmax_j( q_i . k_j / sqrt(head_dim) ) v_j
+ * written at token i's original grid position. Softmax statistics and
+ * accumulators are float32; with BASA_BF16 the products run on the tensor
+ * cores in bfloat16 and the output is rounded once to bfloat16.
+ * kp, vp must be NULL iff the pool patch is all zero; route_idx must be NULL
+ * iff routed_k == 0. Route ids must lie in [0, nWin) (not checked on device).
+ * bfloat16 requires head_dim == 128; float32 supports 64 and 128.
+ */
+basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v,
+                                 const void *kp, const void *vp,
+                                 const int32_t *route_idx, void *out,
+                                 const basa_params *p, basa_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *basa_status_string(basa_status s);
+
+/* Map a device error word (read back from basa_params.dev_err) to a status:
+ * 0 -> BASA_OK, any BASA_DEVERR_TIMEOUT_* bit -> BASA_ERR_DEVICE_TIMEOUT. */
+basa_status basa_device_error_status(int32_t dev_err_word);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASA_H */

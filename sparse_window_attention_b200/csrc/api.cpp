@@ -1,0 +1,114 @@
+// C ABI of libbasa: argument checks, then dispatch to the kernel launchers.
+// Every check runs on the host before any CUDA call, so an invalid call
+// returns its status and launches nothing.
+#include <cstdint>
+#include <cstring>
+
+#include "basa_internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool empty_batch(const basa_params *p) { return p->B == 0 || p->heads == 0; }
+
+// Checks shared by every entry point.
+basa_status check_common(const basa_params *p) {
+  if (!p) return BASA_ERR_INVALID_ARG;
+  if (p->B < 0 || p->heads < 0 || p->n_text < 0 || p->routed_k < 0) return BASA_ERR_INVALID_ARG;
+  if (p->dtype != BASA_BF16 && p->dtype != BASA_F32) return BASA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (p->T < 1 || p->H < 1 || p->W < 1) return BASA_ERR_SHAPE;
+  if (p->wt < 1 || p->wh < 1 || p->ww < 1) return BASA_ERR_SHAPE;
+  if (p->T % p->wt || p->H % p->wh || p->W % p->ww) return BASA_ERR_SHAPE;
+  if (p->st < 0 || p->st >= p->T || p->sy < 0 || p->sy >= p->H || p->sx < 0 || p->sx >= p->W) return BASA_ERR_SHAPE;
+  const bool no_pool = p->pt == 0 && p->ph == 0 && p->pw == 0;
+  if (!no_pool) {
+    if (p->pt < 1 || p->ph < 1 || p->pw < 1) return BASA_ERR_SHAPE;
+    if (p->T % p->pt || p->H % p->ph || p->W % p->pw) return BASA_ERR_SHAPE;
+  }
+  const int64_t N = int64_t(p->T) * p->H * p->W;
+  const int64_t rows = N + p->n_text;
+  if (rows >= (int64_t(1) << 31)) return BASA_ERR_UNSUPPORTED;
+  const int64_t bh = int64_t(p->B) * p->heads;
+  if (bh >= (int64_t(1) << 31)) return BASA_ERR_UNSUPPORTED;
+  const int64_t nwin = N / (int64_t(p->wt) * p->wh * p->ww);
+  if (p->routed_k > 0) {
+    if (p->routed_k > basa::kMaxRouted || p->routed_k > nwin - 1) return BASA_ERR_INVALID_ARG;
+  }
+  return BASA_OK;
+}
+
+bool has_pool(const basa_params *p) { return p->pt > 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char *basa_status_string(basa_status s) {
+  switch (s) {
+    case BASA_OK: return "BASA_OK";
+    case BASA_ERR_INVALID_ARG: return "BASA_ERR_INVALID_ARG";
+    case BASA_ERR_SHAPE: return "BASA_ERR_SHAPE";
+    case BASA_ERR_UNSUPPORTED: return "BASA_ERR_UNSUPPORTED";
+    case BASA_ERR_CUDA: return "BASA_ERR_CUDA";
+    case BASA_ERR_DEVICE_TIMEOUT: return "BASA_ERR_DEVICE_TIMEOUT";
+  }
+  return "BASA_ERR_UNKNOWN";
+}
+
+basa_status basa_device_error_status(int32_t w) {
+  return w == 0 ? BASA_OK : BASA_ERR_DEVICE_TIMEOUT;
+}
+
+basa_status basa_pool_kv(const void *k, const void *v, void *kp, void *vp, const basa_params *p,
+                         basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (!has_pool(p)) return BASA_ERR_INVALID_ARG;
+  if (empty_batch(p)) return BASA_OK;
+  if (!k || !v || !kp || !vp) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kp) || !aligned16(vp)) return BASA_ERR_INVALID_ARG;
+  return basa::launch_pool_kv(k, v, kp, vp, *p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t basa_route_workspace_bytes(const basa_params *p) {
+  if (check_common(p) != BASA_OK) return 0;
+  const size_t nwin = size_t(p->T / p->wt) * (p->H / p->wh) * (p->W / p->ww);
+  return 2 * size_t(p->B) * p->heads * nwin * p->head_dim * sizeof(float);
+}
+
+basa_status basa_route_windows(const void *q, const void *k, int32_t *route_idx, float *route_score,
+                               void *workspace, const basa_params *p, basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (p->routed_k < 1) return BASA_ERR_INVALID_ARG;
+  const int64_t nwin = int64_t(p->T / p->wt) * (p->H / p->wh) * (p->W / p->ww);
+  if (nwin > 4096) return BASA_ERR_UNSUPPORTED;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q || !k || !route_idx || !workspace) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned4(route_idx)) return BASA_ERR_INVALID_ARG;
+  if (route_score && !aligned4(route_score)) return BASA_ERR_INVALID_ARG;
+  return basa::launch_route(q, k, route_idx, route_score, workspace, *p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                                 const int32_t *route_idx, void *out, const basa_params *p,
+                                 basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (p->dtype == BASA_BF16 && p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q || !k || !v || !out) return BASA_ERR_INVALID_ARG;
+  if (has_pool(p) != (kp != nullptr) || has_pool(p) != (vp != nullptr)) return BASA_ERR_INVALID_ARG;
+  if ((p->routed_k > 0) != (route_idx != nullptr)) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return BASA_ERR_INVALID_ARG;
+  if (kp && (!aligned16(kp) || !aligned16(vp))) return BASA_ERR_INVALID_ARG;
+  if (route_idx && !aligned4(route_idx)) return BASA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == BASA_F32) return basa::launch_attn_f32(q, k, v, kp, vp, route_idx, out, *p, s);
+  return basa::launch_attn_bf16(q, k, v, kp, vp, route_idx, out, *p, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// Internal declarations shared by the host layer and the kernels of libbasa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/basa.h"
+
+namespace basa {
+
+// ---------------------------------------------------------------------------
+// Window tiling plan of the tensor-core attention kernel.
+//
+// A window of the shifted grid is, in the original grid, an axis-aligned block
+// that wraps around the grid edge in every axis whose shift is not a multiple
+// of the window extent. Along such an axis it splits into two contiguous parts
+// (lengths a and w - a, a = w - (s mod w)); all windows share the same split,
+// so a window is one of at most 8 "types" (wrap in t / y / x or not).
+//
+// For each type the host cuts the window into "pieces": boxes of at most 128
+// tokens that lie inside one part per axis, so each piece is ONE TMA box load
+// (the cyclic shift costs no copy, only coordinate arithmetic). Pieces are
+// packed into 128-row tiles at 8-row (1024-byte) aligned offsets, which keeps
+// every TMA destination aligned to the 128-byte swizzle atom. The same tiles
+// serve as query tiles (M = 128 rows of the MMA) and as key/value tiles.
+// ---------------------------------------------------------------------------
+constexpr int kTileRows = 128;
+constexpr int kMaxShapes = 8;
+constexpr int kMaxPieces = 256;
+constexpr int kMaxTiles = 128;
+constexpr int kMaxRouted = 16;
+
+struct PlanShape {
+  int16_t ct, cy, cx, rows;  // box extents in t, y, x and their product
+};
+
+struct PlanPiece {
+  int16_t lt, ly, lx;  // offset of the piece inside the window (window-local coordinates)
+  uint8_t shape;       // index into WindowPlan::shape
+  uint8_t dest;        // first row of the piece inside its tile (multiple of 8)
+};
+
+struct PlanTile {
+  uint16_t first_piece, n_pieces;
+  uint16_t valid_rows, pad;
+  uint32_t mask[4];  // bit r set = row r of the tile holds a token
+};
+
+struct PlanType {
+  uint16_t first_tile, n_tiles;
+};
+
+struct WindowPlan {
+  int n_shapes, n_tiles, n_pieces, max_pairs;
+  int zero_fill;  // some tile leaves rows that no TMA load writes
+  PlanShape shape[kMaxShapes];
+  PlanType type[8];
+  PlanTile tile[kMaxTiles];
+  PlanPiece piece[kMaxPieces];
+};
+
+// Builds the plan. Returns BASA_ERR_UNSUPPORTED when a limit above is exceeded.
+basa_status build_window_plan(const basa_params &p, WindowPlan *plan);
+
+// Geometry helpers shared by host and device code.
+struct Geo {
+  int T, H, W, wt, wh, ww, st, sy, sx;
+  int nWt, nWy, nWx, nWin, N;
+};
+
+__host__ __device__ inline Geo make_geo(const basa_params &p) {
+  Geo g;
+  g.T = p.T; g.H = p.H; g.W = p.W;
+  g.wt = p.wt; g.wh = p.wh; g.ww = p.ww;
+  g.st = p.st; g.sy = p.sy; g.sx = p.sx;
+  g.nWt = p.T / p.wt; g.nWy = p.H / p.wh; g.nWx = p.W / p.ww;
+  g.nWin = g.nWt * g.nWy * g.nWx;
+  g.N = p.T * p.H * p.W;
+  return g;
+}
+
+// Origin (original-grid coordinates) of shifted window `w` and its type bits
+// (1 = wraps in t, 2 = wraps in y, 4 = wraps in x).
+__host__ __device__ inline void window_origin(const Geo &g, int w, int *ot, int *oy, int *ox, int *type) {
+  int jx = w % g.nWx;
+  int jy = (w / g.nWx) % g.nWy;
+  int jt = w / (g.nWx * g.nWy);
+  *ot = (jt * g.wt + g.st) % g.T;
+  *oy = (jy * g.wh + g.sy) % g.H;
+  *ox = (jx * g.ww + g.sx) % g.W;
+  *type = (*ot + g.wt > g.T ? 1 : 0) | (*oy + g.wh > g.H ? 2 : 0) | (*ox + g.ww > g.W ? 4 : 0);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (each returns BASA_OK or BASA_ERR_CUDA).
+// ---------------------------------------------------------------------------
+basa_status launch_pool_kv(const void *k, const void *v, void *kp, void *vp, const basa_params &p, cudaStream_t s);
+basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float *route_score, void *workspace,
+                         const basa_params &p, cudaStream_t s);
+basa_status launch_attn_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                            const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
+basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                             const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
+
+}  // namespace basa

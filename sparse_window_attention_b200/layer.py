@@ -1,0 +1,76 @@
+"""One BASA layer call on device tensors: pool -> (route) -> attention.
+
+``BasaLayer`` owns the intermediate device buffers of one layer shape (pooled
+K/V, routed window ids and scores, the routing workspace and the device error
+word), allocated once with torch, and calls the three C entry points on the
+current CUDA stream. It computes nothing itself.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class BasaLayer:
+    def __init__(self, batch, heads, head_dim, grid, window, pool=(0, 0, 0), n_text=0, routed_k=0, dtype="bf16",
+                 device="cuda"):
+        self.batch, self.heads, self.head_dim = batch, heads, head_dim
+        self.grid, self.window, self.pool = tuple(grid), tuple(window), tuple(pool)
+        self.n_text, self.routed_k, self.dtype = n_text, routed_k, dtype
+        self.device = torch.device(device)
+        T, H, W = self.grid
+        self.N = T * H * W
+        self.n_win = (T // window[0]) * (H // window[1]) * (W // window[2])
+        self.has_pool = all(p > 0 for p in self.pool)
+        self.n_pool = (T // pool[0]) * (H // pool[1]) * (W // pool[2]) if self.has_pool else 0
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.kp = self.vp = None
+        if self.has_pool:
+            self.kp = torch.empty(batch, heads, self.n_pool, head_dim, dtype=tdt, device=self.device)
+            self.vp = torch.empty_like(self.kp)
+        self.route_idx = self.route_score = self.workspace = None
+        if routed_k > 0:
+            self.route_idx = torch.empty(batch, heads, self.n_win, routed_k, dtype=torch.int32, device=self.device)
+            self.route_score = torch.empty(batch, heads, self.n_win, routed_k, dtype=torch.float32, device=self.device)
+            nbytes = B.basa_route_workspace_bytes(self.params((0, 0, 0)))
+            self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+        self._params = {}
+
+    def params(self, shift, **extra) -> B.basa_params:
+        key = (tuple(shift), tuple(sorted(extra.items())))
+        if key not in self._params:
+            self._params[key] = B.make_params(self.batch, self.heads, self.head_dim, self.grid, self.window, shift,
+                                              self.pool, self.n_text, self.routed_k, self.dtype,
+                                              dev_err=self.dev_err, **extra)
+        return self._params[key]
+
+    def pool_kv(self, k, v, shift=(0, 0, 0), stream=None):
+        B.basa_pool_kv(k, v, self.kp, self.vp, self.params(shift), stream)
+
+    def route(self, q, k, shift, stream=None):
+        B.basa_route_windows(q, k, self.route_idx, self.route_score, self.workspace, self.params(shift), stream)
+
+    def attention(self, q, k, v, out, shift, kp=None, vp=None, route_idx=None, stream=None, **extra):
+        kp = self.kp if kp is None else kp
+        vp = self.vp if vp is None else vp
+        route_idx = self.route_idx if route_idx is None else route_idx
+        B.basa_window_attn_fwd(q, k, v, kp, vp, route_idx, out, self.params(shift, **extra), stream)
+
+    def forward(self, q, k, v, shift, out=None, stream=None):
+        """Full layer: pooled K/V, routed windows (if routed_k > 0), attention."""
+        if out is None:
+            out = torch.empty_like(q)
+        if self.has_pool:
+            self.pool_kv(k, v, shift, stream)
+        if self.routed_k > 0:
+            self.route(q, k, shift, stream)
+        self.attention(q, k, v, out, shift, stream=stream)
+        return out
+
+    def launches_per_forward(self) -> int:
+        return (1 if self.has_pool else 0) + (2 if self.routed_k > 0 else 0) + 1
+
+    def device_error(self) -> int:
+        return int(self.dev_err.item())

@@ -1,0 +1,108 @@
+"""Host-only checks of the C ABI: the library loads, exports what include/basa.h
+declares, and rejects invalid calls with the documented status before any CUDA
+call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_window_attention_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "basa.h")).read()
+    return sorted(set(re.findall(r"^\w[\w\s\*]*?\b(basa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert set(names) == set(B.EXPORTED), names
+    lib = ctypes.CDLL(os.path.join(ROOT, "sparse_window_attention_b200", "libbasa.so"))
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for code, name in B.STATUS_NAMES.items():
+        assert B.basa_status_string(code) == name
+    assert B.basa_device_error_status(0) == B.BASA_OK
+    assert B.basa_device_error_status(2) == 5
+
+
+def test_params_struct_layout_matches_header():
+    # 18 ints, a pointer, two uint32 -> 72 + 8 + 8 bytes on LP64
+    assert ctypes.sizeof(B.basa_params) == 88
+    assert B.basa_params.dev_err.offset == 72
+
+
+def _p(**kw):
+    base = dict(B=1, heads=2, head_dim=128, grid=(1, 64, 64), window=(1, 16, 16), shift=(0, 8, 8), pool=(1, 8, 8),
+                n_text=16, routed_k=0, dtype="bf16")
+    base.update(kw)
+    return B.make_params(base["B"], base["heads"], base["head_dim"], base["grid"], base["window"], base["shift"],
+                         base["pool"], base["n_text"], base["routed_k"], base["dtype"])
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every case fails its checks first
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(head_dim=96), 3),
+        (dict(grid=(1, 60, 64)), 2),
+        (dict(window=(1, 16, 20)), 2),
+        (dict(shift=(0, 64, 0)), 2),
+        (dict(shift=(0, -1, 0)), 2),
+        (dict(pool=(1, 8, 0)), 2),
+        (dict(pool=(1, 7, 8)), 2),
+        (dict(n_text=-1), 1),
+        (dict(routed_k=16), 1),  # nWin - 1 = 15
+        (dict(routed_k=17, grid=(1, 128, 128)), 1),
+        (dict(B=-1), 1),
+        (dict(dtype=7), 1),
+    ],
+)
+def test_invalid_params_rejected_before_launch(kw, status):
+    p = _p(**kw)
+    if kw.get("dtype") == 7:
+        p.dtype = 7
+    got = B.basa_window_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE if p.routed_k > 0 else None, FAKE, p,
+                                 stream=0, check=False)
+    assert got == status
+
+
+def test_pointer_rules():
+    p = _p()
+    # pooled pointers must be given iff a pool patch is set
+    assert B.basa_window_attn_fwd(FAKE, FAKE, FAKE, None, None, None, FAKE, p, stream=0, check=False) == 1
+    # misaligned
+    assert B.basa_window_attn_fwd(FAKE + 8, FAKE, FAKE, FAKE, FAKE, None, FAKE, p, stream=0, check=False) == 1
+    # null output
+    assert B.basa_window_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, p, stream=0, check=False) == 1
+    # route ids must be given iff routed_k > 0
+    pr = _p(routed_k=2)
+    assert B.basa_window_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, pr, stream=0, check=False) == 1
+    assert B.basa_window_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, p, stream=0, check=False) == 1
+    # bfloat16 attention is built for head_dim 128 only
+    assert B.basa_window_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, _p(head_dim=64), stream=0, check=False) == 3
+    # pooling needs a patch; routing needs routed_k >= 1
+    assert B.basa_pool_kv(FAKE, FAKE, FAKE, FAKE, _p(pool=(0, 0, 0)), stream=0, check=False) == 1
+    assert B.basa_route_windows(FAKE, FAKE, FAKE, None, FAKE, p, stream=0, check=False) == 1
+    assert B.basa_route_windows(FAKE, FAKE, FAKE + 2, None, FAKE, pr, stream=0, check=False) == 1
+
+
+def test_empty_batch_is_a_no_op():
+    for kw in (dict(B=0), dict(heads=0)):
+        p = _p(**kw)
+        assert B.basa_window_attn_fwd(None, None, None, None, None, None, None, p, stream=0, check=False) == 0
+        assert B.basa_pool_kv(None, None, None, None, p, stream=0, check=False) == 0
+
+
+def test_route_workspace_bytes():
+    p = _p(routed_k=2)
+    assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4
+    assert B.basa_route_workspace_bytes(_p(head_dim=100)) == 0

@@ -1,0 +1,40 @@
+"""Failure detection without a GPU fault: a test hook makes the attention
+kernel's loader skip the first key tile, so every wait on it runs into its
+(short) time limit; the kernel records the expiry in the device error word,
+frees its resources and returns. The context must stay usable."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import basa_oracle as O
+from sparse_window_attention_b200 import synth
+from tests import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_expires_and_context_survives():
+    from sparse_window_attention_b200 import binding as B
+    from sparse_window_attention_b200.layer import BasaLayer
+
+    wl = synth.Workload("timeout", "bf16", 1, 2, 128, (1, 32, 32), (1, 16, 16), (0, 8, 8), (1, 8, 8), 0, 0, "iid")
+    (q, k, v), (qd, kd, vd) = PT.gpu_inputs(wl)
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    out = torch.zeros_like(qd)
+    layer.pool_kv(kd, vd, wl.shift)
+    layer.attention(qd, kd, vd, out, wl.shift, flags=B.BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD, wait_timeout_us=20000)
+    torch.cuda.synchronize()
+    err = layer.device_error()
+    assert err & 0x2, f"the MMA issuer's wait on the missing tile should expire (word {err:#x})"
+    assert B.basa_device_error_status(err) == 5
+    assert B.basa_status_string(B.basa_device_error_status(err)) == "BASA_ERR_DEVICE_TIMEOUT"
+    # no output was stored
+    assert torch.count_nonzero(out).item() == 0
+    # the context is still usable: a normal call matches the oracle
+    layer.dev_err.zero_()
+    out2 = layer.forward(qd, kd, vd, wl.shift)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    geo = PT.geometry(wl)
+    ref = O.basa_attention(PT.to64(q), PT.to64(k), PT.to64(v), geo)
+    PT.assert_outputs_close(PT.to64(out2), ref, "bf16", "after timeout")
