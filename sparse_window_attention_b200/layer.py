@@ -25,6 +25,7 @@ class BasaLayer:
         self.has_pool = all(p > 0 for p in self.pool)
         self.n_pool = (T // pool[0]) * (H // pool[1]) * (W // pool[2]) if self.has_pool else 0
         tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self._params = {}
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.kp = self.vp = None
         if self.has_pool:
@@ -36,7 +37,6 @@ class BasaLayer:
             self.route_score = torch.empty(batch, heads, self.n_win, routed_k, dtype=torch.float32, device=self.device)
             nbytes = B.basa_route_workspace_bytes(self.params((0, 0, 0)))
             self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
-        self._params = {}
 
     def params(self, shift, **extra) -> B.basa_params:
         key = (tuple(shift), tuple(sorted(extra.items())))
