@@ -149,6 +149,38 @@ basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v,
                                  const int32_t *route_idx, void *out,
                                  const basa_params *p, basa_stream_t stream);
 
+/*
+ * basa_route_windows_noalloc — basa_route_windows without a caller workspace.
+ * The paper has no counterpart: this is a library convenience.
+ *
+ * For callers that cannot allocate device memory at the point of the call: a
+ * plain C host with no allocator object to carve a workspace from, a plugin in a
+ * framework whose caching allocator owns the device memory (a private
+ * cudaMalloc can fail or fragment its pool), or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not allowed. Same operation,
+ * arguments and results as basa_route_windows, minus `workspace`; the window
+ * means go to a fixed scratch array of BASA_NOALLOC_SCRATCH_BYTES (4 MiB) that
+ * lives in the library's device image: every GPU that loads the library holds
+ * it until the process exits.
+ *
+ * Limits and caveats:
+ *  - basa_route_workspace_bytes(p) must be <= BASA_NOALLOC_SCRATCH_BYTES, else
+ *    BASA_ERR_UNSUPPORTED is returned and nothing is launched (e.g. Wan-shaped
+ *    12 heads x 140 windows x 128 needs 1.7 MiB).
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero). Calls whose kernels
+ *    overlap on the GPU (different streams, no ordering between them) race on
+ *    it; order them on one stream or with events.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define BASA_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+basa_status basa_route_windows_noalloc(const void *q, const void *k, int32_t *route_idx,
+                                       float *route_score, const basa_params *p,
+                                       basa_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *basa_status_string(basa_status s);
 

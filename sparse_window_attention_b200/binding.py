@@ -29,6 +29,7 @@ EXPORTED = (
     "basa_pool_kv",
     "basa_route_workspace_bytes",
     "basa_route_windows",
+    "basa_route_windows_noalloc",
     "basa_window_attn_fwd",
     "basa_status_string",
     "basa_device_error_status",
@@ -68,6 +69,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.basa_route_workspace_bytes.restype = ctypes.c_size_t
     lib.basa_route_windows.argtypes = [vp, vp, vp, vp, vp, P, vp]
     lib.basa_route_windows.restype = ctypes.c_int
+    lib.basa_route_windows_noalloc.argtypes = [vp, vp, vp, vp, P, vp]
+    lib.basa_route_windows_noalloc.restype = ctypes.c_int
     lib.basa_window_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, P, vp]
     lib.basa_window_attn_fwd.restype = ctypes.c_int
     lib.basa_status_string.argtypes = [ctypes.c_int]
@@ -141,6 +144,16 @@ def basa_route_windows(q, k, route_idx, route_score, workspace, params: basa_par
                                  ctypes.byref(params), _stream(stream))
     if check:
         _check(st, "basa_route_windows")
+    return st
+
+
+def basa_route_windows_noalloc(q, k, route_idx, route_score, params: basa_params, stream=None, check=True) -> int:
+    """basa_route_windows without a workspace argument (uses the library's fixed
+    device scratch; see include/basa.h for its limits)."""
+    st = _lib.basa_route_windows_noalloc(_ptr(q), _ptr(k), _ptr(route_idx), _ptr(route_score),
+                                         ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_route_windows_noalloc")
     return st
 
 

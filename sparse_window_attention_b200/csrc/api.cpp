@@ -93,6 +93,21 @@ basa_status basa_route_windows(const void *q, const void *k, int32_t *route_idx,
   return basa::launch_route(q, k, route_idx, route_score, workspace, *p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+basa_status basa_route_windows_noalloc(const void *q, const void *k, int32_t *route_idx, float *route_score,
+                                       const basa_params *p, basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (p->routed_k < 1) return BASA_ERR_INVALID_ARG;
+  const int64_t nwin = int64_t(p->T / p->wt) * (p->H / p->wh) * (p->W / p->ww);
+  if (nwin > 4096) return BASA_ERR_UNSUPPORTED;
+  if (basa_route_workspace_bytes(p) > BASA_NOALLOC_SCRATCH_BYTES) return BASA_ERR_UNSUPPORTED;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q || !k || !route_idx) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned4(route_idx)) return BASA_ERR_INVALID_ARG;
+  if (route_score && !aligned4(route_score)) return BASA_ERR_INVALID_ARG;
+  return basa::launch_route_noalloc(q, k, route_idx, route_score, *p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                                  const int32_t *route_idx, void *out, const basa_params *p,
                                  basa_stream_t stream) {

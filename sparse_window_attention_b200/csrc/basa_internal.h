@@ -98,6 +98,9 @@ __host__ __device__ inline void window_origin(const Geo &g, int w, int *ot, int 
 basa_status launch_pool_kv(const void *k, const void *v, void *kp, void *vp, const basa_params &p, cudaStream_t s);
 basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float *route_score, void *workspace,
                          const basa_params &p, cudaStream_t s);
+// Routing with the library's fixed device scratch array instead of a workspace.
+basa_status launch_route_noalloc(const void *q, const void *k, int32_t *route_idx, float *route_score,
+                                 const basa_params &p, cudaStream_t s);
 basa_status launch_attn_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                             const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,

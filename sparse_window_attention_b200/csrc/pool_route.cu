@@ -12,6 +12,7 @@
 
 #include <cfloat>
 #include <climits>
+#include <mutex>
 
 #include "basa_internal.h"
 
@@ -237,6 +238,39 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
   const int ngroups = (g.nWin + kRouteWarps - 1) / kRouteWarps;
   route_topk_kernel<<<unsigned(bh) * unsigned(ngroups), kRouteWarps * 32, smem, s>>>(r);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- no-allocation routing
+// Window-mean scratch for basa_route_windows_noalloc, for callers that cannot
+// allocate device memory themselves. It is part of the library's device image,
+// so every GPU that loads the library holds it until the process exits. In host
+// code `g_route_scratch` names a host-side stand-in, not a device address: the
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_route_scratch[BASA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxScratchDevices] = {};
+}  // namespace
+
+basa_status launch_route_noalloc(const void *q, const void *k, int32_t *route_idx, float *route_score,
+                                 const basa_params &p, cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BASA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxScratchDevices) return BASA_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+      // `dev` is the current device here, so this is the address on that device.
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_route_scratch) != cudaSuccess || !addr) return BASA_ERR_CUDA;
+      g_scratch_addr[dev] = addr;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  return launch_route(q, k, route_idx, route_score, scratch, p, s);
 }
 
 }  // namespace basa
