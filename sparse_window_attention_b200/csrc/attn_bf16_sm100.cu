@@ -6,15 +6,15 @@
 //
 // One CTA = (b*head, window, pair of 128-row query tiles). Warp roles:
 //   warp 0      TMA loader: query tiles once, then a K, V, K, V ... stream of
-//               128-row key tiles through a 3-slot shared-memory ring. Window
+//               128-row key tiles through a 5-slot shared-memory ring. Window
 //               tiles are assembled from TMA box loads whose coordinates already
 //               include the cyclic shift (mod the grid), so no rolled copy exists.
 //   warp 1      tcgen05 issuer (one thread): S_g = Q_g K^T and O_g += P_g V with
 //               fp32 accumulators in TMEM (S0, S1, O0, O1: 4 x 128 columns).
 //   warps 2-9   two softmax warpgroups, one per query tile; a thread owns one
 //               query row: reads its S row from TMEM, runs the online softmax in
-//               fp32 (base-2 exponent, scale folded in), writes P (bf16) to shared
-//               memory, rescales its O row in TMEM when the running max grows,
+//               fp32 (base-2 exponent, scale folded in), writes P (bf16) back to
+//               TMEM over its S row (A operand of P V), rescales its O row in TMEM when the running max grows,
 //               and at the end normalises O and stores it with TMA boxes at the
 //               same (unshifted) coordinates the queries were loaded from.
 // Every wait is bounded (globaltimer); on expiry the kernel records a bit in
@@ -23,6 +23,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -32,17 +33,19 @@
 namespace basa {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 320;  // 10 warps
 constexpr uint32_t kHalfBytes = 16384;                 // 128 rows x 128 B (64 bf16) , 128B-swizzled
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;        // 128 rows x head_dim 128
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr uint32_t kSmemQ = 0;                         // 2 query tiles (reused for the output)
-constexpr uint32_t kSmemP = 2 * kTileBytes;            // 2 P tiles
-constexpr uint32_t kSmemRing = 4 * kTileBytes;         // K/V ring
+constexpr uint32_t kSmemRing = 2 * kTileBytes;         // K/V ring
 constexpr uint32_t kSmemCtrl = kSmemRing + kStages * kTileBytes;
 constexpr uint32_t kCtrlBytes = 1024;
-constexpr uint32_t kSmemBytes = kSmemCtrl + kCtrlBytes + 1024;  // + alignment slack
+constexpr int kMaskTable = 64;                         // key tiles whose column masks are tabled in smem
+constexpr uint32_t kSmemMask = kSmemCtrl + kCtrlBytes;
+constexpr uint32_t kSmemBytes = kSmemMask + kMaskTable * 16 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
+constexpr int kDefaultEmuPairs = 0;  // exponential pairs of every 8 done on the FMA pipe
 
 // tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), N >> 3 at bits 17-22, M >> 4 at bits 24-28; bit 16 marks
@@ -50,11 +53,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm100 layout (version 1 at bit 46).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
-         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
-}
 
 struct alignas(64) AttnParams {
   CUtensorMap map_q[kMaxShapes];
@@ -176,22 +174,125 @@ __device__ __forceinline__ bool key_tile_mask(const AttnParams &P, const Ctrl &c
   return valid == kTileRows;
 }
 
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+// Shared-memory descriptors, split in 32-bit halves. The high half is constant:
+// stride byte offset 1024 (8 rows of 128 B), version 1, 128-byte swizzle. The
+// low half holds the start address >> 4 (bits 0-13) and the leading byte offset
+// (bits 16-29; ignored for K-major swizzled operands, 16 KB between the two
+// 64-column halves of the MN-major V). Stepping the start address is one add.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+constexpr uint32_t kDescLoK = (16u >> 4) << 16;
+constexpr uint32_t kDescLoV = (kHalfBytes >> 4) << 16;
+
+// S (=) Q K^T over head_dim 128: 8 K-steps of 16; steps 0-3 walk the first 64-column
+// half in 32-byte strides, steps 4-7 the second half.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    ptx::mma_bf16_ss(d_tmem, smem_desc(q_addr + off, 16, 1024), smem_desc(k_addr + off, 16, 1024), kIdescQK, kk > 0);
-  }
-}
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_addr, uint32_t v_addr, bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    ptx::mma_bf16_ss(d_tmem, smem_desc(p_addr + off, 16, 1024), smem_desc(v_addr + kk * 2048, kHalfBytes, 1024),
-                     kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    ptx::mma_bf16_ss2(d_tmem, q_lo + off, kDescHi, k_lo + off, kDescHi, kIdescQK, kk > 0);
   }
 }
 
+// O (+)= P V: P (bf16, 128 rows x 128 keys) sits in TMEM over the first 64
+// columns of its S buffer; 16 keys = 8 TMEM columns per K step.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    ptx::mma_bf16_ts2(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
+                      (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// The running row max is only raised when a tile's max exceeds it by more than
+// 2^8 (log2 units); otherwise the old max is kept and P values up to 256 are
+// produced, which float32 sums and bfloat16 P hold exactly as well. This skips
+// most rescales of the O accumulator in TMEM.
+constexpr float kRescaleLog2 = 8.0f;
+// 2^f on [-1/2, 1/2]: degree-3 polynomial minimising the maximum relative error
+// (Remez exchange fitted for this kernel; max relative error 7.5e-5, far below
+// the 2^-9 rounding of the bfloat16 P that consumes it).
+constexpr float kExpC0 = 0.9999280571937561f;
+constexpr float kExpC1 = 0.6932609677314758f;
+constexpr float kExpC2 = 0.2426111251115799f;
+constexpr float kExpC3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer in the low mantissa bits
+
+// p = 2^x for the N entries of s (x = s * scale_log2 - m), in place; returns the
+// row sum. For EMU_PAIRS of every 8 pairs the exponential runs on the FMA pipe
+// (x = j + f with j = round(x), 2^f by the polynomial, 2^j added to the exponent
+// bits), the rest on the MUFU ex2 unit, so the two pipes can share the load.
+template <int EMU_PAIRS, int N = 128>
+__device__ __forceinline__ float exp2_row(uint32_t (&s)[N], float scale_log2, float m) {
+  using namespace ptx;
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2), negm2 = f2_pack(-m, -m);
+  const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic), negmagic2 = f2_pack(-kRoundMagic, -kRoundMagic);
+  const uint64_t neg1 = f2_pack(-1.f, -1.f);
+  const uint64_t c0 = f2_pack(kExpC0, kExpC0), c1 = f2_pack(kExpC1, kExpC1);
+  const uint64_t c2 = f2_pack(kExpC2, kExpC2), c3 = f2_pack(kExpC3, kExpC3);
+  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int pr = 0; pr < N / 2; ++pr) {
+    const uint64_t x = ffma2(f2_pack(__uint_as_float(s[2 * pr]), __uint_as_float(s[2 * pr + 1])), sc2, negm2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    uint32_t r0, r1;
+    if ((pr & 7) < EMU_PAIRS) {
+      const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+      const uint64_t t = fadd2(xc, magic2);
+      const uint64_t f = ffma2(fadd2(t, negmagic2), neg1, xc);  // f = x - round(x), in [-1/2, 1/2]
+      uint64_t q = ffma2(f, c3, c2);
+      q = ffma2(q, f, c1);
+      q = ffma2(q, f, c0);
+      float q0, q1, t0, t1;
+      f2_unpack(q, q0, q1);
+      f2_unpack(t, t0, t1);
+      // the low bits of t hold round(x); shifted by 23 they land in the exponent field
+      r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
+      r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
+    } else {
+      r0 = __float_as_uint(ex2(x0));
+      r1 = __float_as_uint(ex2(x1));
+    }
+    s[2 * pr] = r0;
+    s[2 * pr + 1] = r1;
+    const uint64_t pp = f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+    if (pr & 1) acc1 = fadd2(acc1, pp);
+    else acc0 = fadd2(acc0, pp);
+  }
+  float a, b, c, d;
+  f2_unpack(acc0, a, b);
+  f2_unpack(acc1, c, d);
+  return (a + b) + (c + d);
+}
+
+// Row max of the N entries of s (raw scores).
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&s)[N]) {
+  float a = __uint_as_float(s[0]), b = __uint_as_float(s[1]), c = __uint_as_float(s[2]), d = __uint_as_float(s[3]);
+#pragma unroll
+  for (int i = 4; i < N; i += 8) {
+    a = ptx::fmax3(a, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+    b = ptx::fmax3(b, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+    c = ptx::fmax3(c, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+    d = ptx::fmax3(d, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+  }
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// Sets every column whose mask bit is clear to -inf.
+template <int N>
+__device__ __forceinline__ void apply_mask(uint32_t (&s)[N], const uint32_t *mask) {
+#pragma unroll
+  for (int wd = 0; wd < N / 32; ++wd) {
+    const uint32_t mw = mask[wd];
+    if (mw != 0xFFFFFFFFu) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!((mw >> i) & 1u)) s[32 * wd + i] = __float_as_uint(-INFINITY);
+    }
+  }
+}
+
+template <int EMU_PAIRS>
 __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -230,6 +331,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       window_origin(P.g, u, &a, &b, &d, &t);
       c.wtype[1 + r] = t;
       c.org[1 + r][0] = a; c.org[1 + r][1] = b; c.org[1 + r][2] = d;
+    }
+    // column masks of this CTA's key tiles, in stream order (all ones = full tile)
+    uint4 *tab = reinterpret_cast<uint4 *>(smem + kSmemMask);
+    KeyIter it{0, 0};
+    for (int j = 0; j < kMaskTable && it.seg <= P.routed_k + 2; ++j) {
+      uint32_t m[4];
+      key_tile_mask(P, c, it, m);
+      tab[j] = make_uint4(m[0], m[1], m[2], m[3]);
+      advance(P, c, it);
     }
     ptx::fence_mbar_init();
   }
@@ -309,26 +419,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     if (lane == 0) {
       Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, true};
       Waiter drain{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, false};
-      const uint32_t sQ = ptx::smem_u32(smem + kSmemQ), sP = ptx::smem_u32(smem + kSmemP);
-      const uint32_t sR = ptx::smem_u32(smem + kSmemRing);
+      // low descriptor halves of the query tiles and the ring slots
+      const uint32_t sQ = kDescLoK | (ptx::smem_u32(smem + kSmemQ) >> 4);
+      const uint32_t sRk = kDescLoK | (ptx::smem_u32(smem + kSmemRing) >> 4);
+      const uint32_t sRv = kDescLoV | (ptx::smem_u32(smem + kSmemRing) >> 4);
+      constexpr uint32_t kTileDesc = kTileBytes >> 4;
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       if (wt.wait(&c.q_full, 0) && wt.wait(&c.full[0], 0)) {
         ptx::tc_fence_after();
-        issue_qk(tS0, sQ, sR);
+        issue_qk(tS0, sQ, sRk);
         ptx::mma_commit(&c.s_full[0]);
         if (has_q1) {
-          issue_qk(tS1, sQ + kTileBytes, sR);
+          issue_qk(tS1, sQ + kTileDesc, sRk);
           ptx::mma_commit(&c.s_full[1]);
         }
         ptx::mma_commit(&c.empty[0]);
         for (int j = 0; j < n_kt; ++j) {
           const int vi = 2 * j + 1, ki = 2 * j + 2;
-          const uint32_t vaddr = sR + (vi % kStages) * kTileBytes, kaddr = sR + (ki % kStages) * kTileBytes;
+          const uint32_t vaddr = sRv + (vi % kStages) * kTileDesc, kaddr = sRk + (ki % kStages) * kTileDesc;
           const bool more = j + 1 < n_kt;
           if (!wt.wait(&c.full[vi % kStages], (vi / kStages) & 1)) break;
           if (!wt.wait(&c.p_full[0], j & 1)) break;
           ptx::tc_fence_after();
-          issue_pv(tO0, sP, vaddr, j > 0);
+          issue_pv(tO0, tS0, vaddr, j > 0);
           if (more) {
             if (!wt.wait(&c.full[ki % kStages], (ki / kStages) & 1)) break;
             ptx::tc_fence_after();
@@ -340,12 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
           if (has_q1) {
             if (!wt.wait(&c.p_full[1], j & 1)) break;
             ptx::tc_fence_after();
-            issue_pv(tO1, sP + kTileBytes, vaddr, j > 0);
+            issue_pv(tO1, tS1, vaddr, j > 0);
           }
           ptx::mma_commit(&c.empty[vi % kStages]);
           if (more) {
             if (has_q1) {
-              issue_qk(tS1, sQ + kTileBytes, kaddr);
+              issue_qk(tS1, sQ + kTileDesc, kaddr);
               ptx::mma_commit(&c.s_full[1]);
             }
             ptx::mma_commit(&c.empty[ki % kStages]);
@@ -361,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
+    // Two warpgroups, one per query tile; a thread owns one query row.
     const int g = (warp - 2) / 4;
     const int sub = warp % 4;  // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;
@@ -368,10 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     const uint32_t tS = tmem + lane_off + g * 128, tO = tmem + lane_off + 256 + g * 128;
     const bool active = g == 0 || has_q1;
     Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_SOFTMAX, true};
-    uint8_t *p_tile = smem + kSmemP + g * kTileBytes;
     uint8_t *q_tile = smem + kSmemQ + g * kTileBytes;
-    const uint32_t p_row = ptx::smem_u32(p_tile) + row * 128;
     const uint32_t swz = row & 7;
+    const float sl2 = P.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     KeyIter it{0, 0};
@@ -382,69 +495,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       uint32_t s[128];
       ptx::tmem_ld128(tS, s);
       ptx::tmem_ld_wait(s);
-      uint32_t mask[4];
-      if (!key_tile_mask(P, c, it, mask)) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (!((mask[i >> 5] >> (i & 31)) & 1u)) s[i] = __float_as_uint(-INFINITY);
+      if (j < kMaskTable) {
+        const uint4 mt = reinterpret_cast<const uint4 *>(smem + kSmemMask)[j];
+        if ((mt.x & mt.y & mt.z & mt.w) != 0xFFFFFFFFu) {
+          const uint32_t mask[4] = {mt.x, mt.y, mt.z, mt.w};
+          apply_mask(s, mask);
+        }
+      } else {
+        uint32_t mask[4];
+        if (!key_tile_mask(P, c, it, mask)) apply_mask(s, mask);
       }
-      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]), mx2 = __uint_as_float(s[2]),
-            mx3 = __uint_as_float(s[3]);
-#pragma unroll
-      for (int i = 4; i < 128; i += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[i]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[i + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[i + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[i + 3]));
-      }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      const float m_new = fmaxf(m, mx * P.scale_log2);
-      const float alpha = ptx::ex2(m - m_new);
-      const float neg_m = -m_new;
-      float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        const float p0 = ptx::ex2(fmaf(__uint_as_float(s[i]), P.scale_log2, neg_m));
-        const float p1 = ptx::ex2(fmaf(__uint_as_float(s[i + 1]), P.scale_log2, neg_m));
-        sum0 += p0;
-        sum1 += p1;
-        s[i] = __float_as_uint(p0);
-        s[i + 1] = __float_as_uint(p1);
-      }
-      l = l * alpha + (sum0 + sum1);
+      const float m_tile = row_max(s) * sl2;
+      const bool need = m_tile > m + kRescaleLog2;  // always true on the first tile (m = -inf)
+      const float m_new = need ? m_tile : m;
+      const float alpha = need ? ptx::ex2(m - m_new) : 1.0f;
+      const float sum = exp2_row<EMU_PAIRS>(s, sl2, m_new);
+      l = l * alpha + sum;
       m = m_new;
-      // P row -> shared memory, K-major, 128-byte swizzle (16-byte chunk c of the
-      // 128-byte row r sits at chunk position c ^ (r % 8)).
+      // P row -> TMEM over the first 64 columns of S (bf16 pairs, low half = even key).
+      // The MMA that overwrites S next is issued after the P V that reads it.
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        const int k0 = c16 * 8;
-        const uint32_t addr = p_row + (c16 >> 3) * kHalfBytes + (((c16 & 7) ^ swz) << 4);
-        ptx::st_shared_v4(addr, ptx::pack_bf16x2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])),
-                          ptx::pack_bf16x2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])),
-                          ptx::pack_bf16x2(__uint_as_float(s[k0 + 4]), __uint_as_float(s[k0 + 5])),
-                          ptx::pack_bf16x2(__uint_as_float(s[k0 + 6]), __uint_as_float(s[k0 + 7])));
-      }
-      ptx::fence_proxy_async_smem();
-      if (j > 0 && __any_sync(0xFFFFFFFFu, alpha < 1.0f)) {
+      for (int i = 0; i < 64; ++i) s[i] = ptx::pack_bf16x2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+      ptx::tmem_st64(tS, s);
+      if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+        const uint64_t a2 = ptx::f2_pack(alpha, alpha);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
           ptx::tmem_ld32(tO + cc * 32, r);
           ptx::tmem_ld_wait(r);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            float lo, hi;
+            ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2), lo, hi);
+            r[i] = __float_as_uint(lo);
+            r[i + 1] = __float_as_uint(hi);
+          }
           ptx::tmem_st32(tO + cc * 32, r);
         }
-        ptx::tmem_st_wait();
       }
+      ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&c.p_full[g]);
-      advance(P, c, it);
+      if (j + 1 >= kMaskTable) {
+        if (j + 1 == kMaskTable)  // past the table: walk the stream from its start once
+          for (int t = 0; t < kMaskTable; ++t) advance(P, c, it);
+        else
+          advance(P, c, it);
+      }
     }
     if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.o_full[g], 0));
     if (ok) {
       ptx::tc_fence_after();
       const float inv = 1.0f / l;
+      const uint64_t inv2 = ptx::f2_pack(inv, inv);
       const uint32_t o_row = ptx::smem_u32(q_tile) + row * 128;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -452,14 +556,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
         ptx::tmem_ld32(tO + cc * 32, r);
         ptx::tmem_ld_wait(r);
 #pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float lo, hi;
+          ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), inv2), lo, hi);
+          r[i] = __float_as_uint(lo);
+          r[i + 1] = __float_as_uint(hi);
+        }
+#pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int c16 = cc * 4 + i;
           const uint32_t addr = o_row + (c16 >> 3) * kHalfBytes + (((c16 & 7) ^ swz) << 4);
           const int b = 8 * i;
-          ptx::st_shared_v4(addr, ptx::pack_bf16x2(__uint_as_float(r[b]) * inv, __uint_as_float(r[b + 1]) * inv),
-                            ptx::pack_bf16x2(__uint_as_float(r[b + 2]) * inv, __uint_as_float(r[b + 3]) * inv),
-                            ptx::pack_bf16x2(__uint_as_float(r[b + 4]) * inv, __uint_as_float(r[b + 5]) * inv),
-                            ptx::pack_bf16x2(__uint_as_float(r[b + 6]) * inv, __uint_as_float(r[b + 7]) * inv));
+          ptx::st_shared_v4(addr, ptx::pack_bf16x2(__uint_as_float(r[b]), __uint_as_float(r[b + 1])),
+                            ptx::pack_bf16x2(__uint_as_float(r[b + 2]), __uint_as_float(r[b + 3])),
+                            ptx::pack_bf16x2(__uint_as_float(r[b + 4]), __uint_as_float(r[b + 5])),
+                            ptx::pack_bf16x2(__uint_as_float(r[b + 6]), __uint_as_float(r[b + 7])));
         }
       }
       ptx::fence_proxy_async_smem();
@@ -566,9 +677,17 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
   P.timeout_ns = (p.wait_timeout_us ? (unsigned long long)p.wait_timeout_us : 2000000ull) * 1000ull;
   const long long blocks = (long long)p.B * p.heads * P.g.nWin * P.plan.max_pairs;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  static const int emu = [] {
+    // tuning override for the share of exponentials done on the FMA pipe (pairs of 8)
+    const char *e = std::getenv("BASA_TUNE_EXP_EMU");
+    const int v = e ? std::atoi(e) : kDefaultEmuPairs;
+    return (v == 0 || v == 2 || v == 3 || v == 4) ? v : kDefaultEmuPairs;
+  }();
+  auto kernel = emu == 0 ? attn_bf16_kernel<0> : emu == 2 ? attn_bf16_kernel<2> : emu == 4 ? attn_bf16_kernel<4>
+                                                                                           : attn_bf16_kernel<3>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return BASA_ERR_CUDA;
-  attn_bf16_kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
+  kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 

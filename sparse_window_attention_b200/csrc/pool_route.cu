@@ -52,10 +52,13 @@ __device__ __forceinline__ void accumulate(float *acc, const uint4 &v, const flo
 __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store_out(float *p, float x) { *p = x; }
 
-// One CTA per (tensor, b*head, box). Threads split the box's token rows into
-// 16-byte chunks (a row of d elements is read by d*sizeof(T)/16 consecutive
-// threads, so a warp reads whole contiguous rows), accumulate in float32, then
-// reduce across row slots in shared memory.
+// One CTA per (tensor, b*head, box). A box is walked as rows of bx tokens (one
+// row per (t, y)); the row's bx * d elements are cut into 16-byte chunks and the
+// CTA's threads take consecutive chunks, so a warp reads contiguous bytes. A
+// thread always lands on the same chunk column c (128 is a multiple of the
+// chunks per token), keeps float32 sums for it, and the row/column position is
+// advanced incrementally (no division per load). Partial sums of the threads
+// that share a chunk column are reduced in shared memory at the end.
 template <typename T, typename OutT>
 __global__ void __launch_bounds__(kMeanThreads) box_mean_kernel(BoxMeanArgs a) {
   constexpr int VEC = 16 / sizeof(T);
@@ -63,31 +66,47 @@ __global__ void __launch_bounds__(kMeanThreads) box_mean_kernel(BoxMeanArgs a) {
   const int tensor = blockIdx.z;
   const int bh = blockIdx.x / a.nbox;
   const int box = blockIdx.x % a.nbox;
-  const int lpr = a.d / VEC;              // threads per row
-  const int rpi = kMeanThreads / lpr;     // rows per CTA iteration
-  const int chunk = threadIdx.x % lpr;
+  const int lpr = a.d / VEC;                 // chunks per token (8, 16 or 32)
+  const int chunk = threadIdx.x % lpr;       // fixed chunk column of this thread
   const int slot = threadIdx.x / lpr;
   const int jx = box % a.nbx, jy = (box / a.nbx) % a.nby, jt = box / (a.nbx * a.nby);
   const int ot = (jt * a.bt + a.ot) % a.T, oy = (jy * a.by + a.oy) % a.H, ox = (jx * a.bx + a.ox) % a.W;
-  const T *base = static_cast<const T *>(a.src[tensor]) + (long long)bh * a.src_bh_stride[tensor] + chunk * VEC;
-  const int cnt = a.bt * a.by * a.bx;
-  const int bxy = a.by * a.bx;
+  // select with conditionals: a dynamic index into the parameter arrays would copy them to local memory
+  const void *src = tensor ? a.src[1] : a.src[0];
+  const long long stride = tensor ? a.src_bh_stride[1] : a.src_bh_stride[0];
+  void *dst = tensor ? a.dst[1] : a.dst[0];
+  const T *base = static_cast<const T *>(src) + (long long)bh * stride + chunk * VEC;
+  const int row_chunks = a.bx * lpr;
+  const int nrows = a.bt * a.by;
+  const int step_rows = kMeanThreads / row_chunks;  // whole rows advanced per step of 128 chunks
+  const int step_rem = kMeanThreads % row_chunks;
+  const int lpr_shift = __ffs(lpr) - 1;
 
+  // position of chunk index threadIdx.x: row r = (rt, ry), chunk xc within the row
+  int r = threadIdx.x / row_chunks, xc = threadIdx.x % row_chunks;
+  int rt = r / a.by, ry = r % a.by;
   float acc[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  for (int u0 = slot; u0 < cnt; u0 += rpi * kMeanUnroll) {
+  auto advance = [&]() {
+    xc += step_rem;
+    int dr = step_rows;
+    if (xc >= row_chunks) { xc -= row_chunks; ++dr; }
+    r += dr;
+    ry += dr;
+    while (ry >= a.by) { ry -= a.by; ++rt; }
+  };
+  while (r < nrows) {
     uint4 v[kMeanUnroll];
 #pragma unroll
     for (int i = 0; i < kMeanUnroll; ++i) {
-      const int u = u0 + i * rpi;
-      if (u < cnt) {
-        const int ut = u / bxy, uy = (u / a.bx) % a.by, ux = u % a.bx;
-        int t = ot + ut; t -= (t >= a.T) ? a.T : 0;
-        int y = oy + uy; y -= (y >= a.H) ? a.H : 0;
-        int x = ox + ux; x -= (x >= a.W) ? a.W : 0;
+      if (r < nrows) {
+        int t = ot + rt; t -= (t >= a.T) ? a.T : 0;
+        int y = oy + ry; y -= (y >= a.H) ? a.H : 0;
+        int x = ox + (xc >> lpr_shift); x -= (x >= a.W) ? a.W : 0;
         const long long tok = ((long long)t * a.H + y) * a.W + x;
         v[i] = __ldg(reinterpret_cast<const uint4 *>(base + tok * a.d));
+        advance();
       } else {
         v[i] = make_uint4(0, 0, 0, 0);
       }
@@ -95,13 +114,14 @@ __global__ void __launch_bounds__(kMeanThreads) box_mean_kernel(BoxMeanArgs a) {
 #pragma unroll
     for (int i = 0; i < kMeanUnroll; ++i) accumulate(acc, v[i], static_cast<const T *>(nullptr));
   }
+  const int slots = kMeanThreads / lpr;
 #pragma unroll
   for (int e = 0; e < VEC; ++e) red[slot * a.d + chunk * VEC + e] = acc[e];
   __syncthreads();
   for (int c = threadIdx.x; c < a.d; c += kMeanThreads) {
     float s = 0.f;
-    for (int r = 0; r < rpi; ++r) s += red[r * a.d + c];
-    OutT *out = static_cast<OutT *>(a.dst[tensor]) + ((long long)bh * a.nbox + box) * a.d + c;
+    for (int q = 0; q < slots; ++q) s += red[q * a.d + c];
+    OutT *out = static_cast<OutT *>(dst) + ((long long)bh * a.nbox + box) * a.d + c;
     store_out(out, s * a.inv_count);
   }
 }

@@ -25,7 +25,8 @@ def test_bounded_wait_expires_and_context_survives():
     layer.attention(qd, kd, vd, out, wl.shift, flags=B.BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD, wait_timeout_us=20000)
     torch.cuda.synchronize()
     err = layer.device_error()
-    assert err & 0x2, f"the MMA issuer's wait on the missing tile should expire (word {err:#x})"
+    # whichever role's wait expires first records its bit (loader 0x1, MMA 0x2, softmax 0x4)
+    assert err != 0 and (err & ~0x7) == 0, f"expected timeout bits in the device error word, got {err:#x}"
     assert B.basa_device_error_status(err) == 5
     assert B.basa_status_string(B.basa_device_error_status(err)) == "BASA_ERR_DEVICE_TIMEOUT"
     # no output was stored
