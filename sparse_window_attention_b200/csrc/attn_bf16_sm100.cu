@@ -216,47 +216,51 @@ constexpr float kExpC2 = 0.2426111251115799f;
 constexpr float kExpC3 = 0.0551716685295105f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer in the low mantissa bits
 
-// p = 2^x for the N entries of s (x = s * scale_log2 - m), in place; returns the
-// row sum. For EMU_PAIRS of every 8 pairs the exponential runs on the FMA pipe
-// (x = j + f with j = round(x), 2^f by the polynomial, 2^j added to the exponent
-// bits), the rest on the MUFU ex2 unit, so the two pipes can share the load.
-template <int EMU_PAIRS, int N = 128>
-__device__ __forceinline__ float exp2_row(uint32_t (&s)[N], float scale_log2, float m) {
+// Which pairs of every 8 take the FMA-pipe exponential, spread evenly so the
+// emulated pairs interleave with MUFU ones: bit k set = pair k (mod 8) emulated.
+__host__ __device__ constexpr uint32_t emu_pair_mask(int n) {
+  return n <= 0 ? 0x00u : n == 1 ? 0x80u : n == 2 ? 0x88u : n == 3 ? 0xA4u : 0xAAu;
+}
+
+// P = 2^x (x = s * scale_log2 - m) for the 128 scores of a row, written in place as
+// the 64 bfloat16 pairs the P V MMA reads (s[i] = pair (2i, 2i+1), low half = even
+// key); each pair is packed as soon as it is computed, so the live register set
+// shrinks along the row. Returns the float32 row sum. For the pairs selected by
+// emu_pair_mask(EMU_PAIRS) the exponential runs on the FMA pipe (x = j + f with
+// j = round(x), 2^f by the polynomial, 2^j added to the exponent bits), the rest
+// on the MUFU ex2 unit.
+template <int EMU_PAIRS>
+__device__ __forceinline__ float exp2_row_packed(uint32_t (&s)[128], float scale_log2, float m) {
   using namespace ptx;
+  constexpr uint32_t kEmu = emu_pair_mask(EMU_PAIRS);
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2), negm2 = f2_pack(-m, -m);
-  const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic), negmagic2 = f2_pack(-kRoundMagic, -kRoundMagic);
-  const uint64_t neg1 = f2_pack(-1.f, -1.f);
-  const uint64_t c0 = f2_pack(kExpC0, kExpC0), c1 = f2_pack(kExpC1, kExpC1);
-  const uint64_t c2 = f2_pack(kExpC2, kExpC2), c3 = f2_pack(kExpC3, kExpC3);
   uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-  for (int pr = 0; pr < N / 2; ++pr) {
+  for (int pr = 0; pr < 64; ++pr) {
     const uint64_t x = ffma2(f2_pack(__uint_as_float(s[2 * pr]), __uint_as_float(s[2 * pr + 1])), sc2, negm2);
     float x0, x1;
     f2_unpack(x, x0, x1);
     uint32_t r0, r1;
-    if ((pr & 7) < EMU_PAIRS) {
+    if ((kEmu >> (pr & 7)) & 1u) {
       const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-      const uint64_t t = fadd2(xc, magic2);
-      const uint64_t f = ffma2(fadd2(t, negmagic2), neg1, xc);  // f = x - round(x), in [-1/2, 1/2]
-      uint64_t q = ffma2(f, c3, c2);
-      q = ffma2(q, f, c1);
-      q = ffma2(q, f, c0);
+      const uint64_t t = fadd2(xc, f2_pack(kRoundMagic, kRoundMagic));
+      const uint64_t f = ffma2(fadd2(t, f2_pack(-kRoundMagic, -kRoundMagic)), f2_pack(-1.f, -1.f), xc);
+      uint64_t q = ffma2(f, f2_pack(kExpC3, kExpC3), f2_pack(kExpC2, kExpC2));
+      q = ffma2(q, f, f2_pack(kExpC1, kExpC1));
+      q = ffma2(q, f, f2_pack(kExpC0, kExpC0));
       float q0, q1, t0, t1;
       f2_unpack(q, q0, q1);
       f2_unpack(t, t0, t1);
-      // the low bits of t hold round(x); shifted by 23 they land in the exponent field
       r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
       r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
     } else {
       r0 = __float_as_uint(ex2(x0));
       r1 = __float_as_uint(ex2(x1));
     }
-    s[2 * pr] = r0;
-    s[2 * pr + 1] = r1;
     const uint64_t pp = f2_pack(__uint_as_float(r0), __uint_as_float(r1));
     if (pr & 1) acc1 = fadd2(acc1, pp);
     else acc0 = fadd2(acc0, pp);
+    s[pr] = pack_bf16x2(__uint_as_float(r0), __uint_as_float(r1));  // s[pr] was read at pair pr / 2
   }
   float a, b, c, d;
   f2_unpack(acc0, a, b);
@@ -509,13 +513,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       const bool need = m_tile > m + kRescaleLog2;  // always true on the first tile (m = -inf)
       const float m_new = need ? m_tile : m;
       const float alpha = need ? ptx::ex2(m - m_new) : 1.0f;
-      const float sum = exp2_row<EMU_PAIRS>(s, sl2, m_new);
+      const float sum = exp2_row_packed<EMU_PAIRS>(s, sl2, m_new);
       l = l * alpha + sum;
       m = m_new;
-      // P row -> TMEM over the first 64 columns of S (bf16 pairs, low half = even key).
-      // The MMA that overwrites S next is issued after the P V that reads it.
-#pragma unroll
-      for (int i = 0; i < 64; ++i) s[i] = ptx::pack_bf16x2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+      // P row -> TMEM over the first 64 columns of S; the MMA that overwrites S
+      // next is issued after the P V that reads it.
       ptx::tmem_st64(tS, s);
       if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
         const uint64_t a2 = ptx::f2_pack(alpha, alpha);
@@ -681,10 +683,11 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
     // tuning override for the share of exponentials done on the FMA pipe (pairs of 8)
     const char *e = std::getenv("BASA_TUNE_EXP_EMU");
     const int v = e ? std::atoi(e) : kDefaultEmuPairs;
-    return (v == 0 || v == 2 || v == 3 || v == 4) ? v : kDefaultEmuPairs;
+    return (v == 0 || v == 2) ? v : kDefaultEmuPairs;
   }();
-  auto kernel = emu == 0 ? attn_bf16_kernel<0> : emu == 2 ? attn_bf16_kernel<2> : emu == 4 ? attn_bf16_kernel<4>
-                                                                                           : attn_bf16_kernel<3>;
+  // Measured on B200 (FLUX 2048^2): every share of FMA-pipe exponentials tried (1/8 to 1/2)
+  // was slower than MUFU only, so 0 is the default; the variant stays for other parts/shapes.
+  auto kernel = emu == 2 ? attn_bf16_kernel<2> : attn_bf16_kernel<0>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return BASA_ERR_CUDA;
   kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
