@@ -160,15 +160,19 @@ def run_ours(args, world, rank, local):
 
     def step(i, ev=None):
         sh = shifts[i % len(shifts)]
+        if ev is not None:
+            ev[0].record(stream)
         if layer.has_pool:
             layer.pool_kv(kd, vd, sh)
+        if ev is not None:
+            ev[1].record(stream)
         if layer.routed_k > 0:
             layer.route(qd, kd, sh)
         if ev is not None:
-            ev[0].record(stream)
+            ev[2].record(stream)
         layer.attention(qd, kd, vd, out, sh)
         if ev is not None:
-            ev[1].record(stream)
+            ev[3].record(stream)
 
     for i in range(args.warmup):
         step(i)
@@ -193,11 +197,13 @@ def run_ours(args, world, rank, local):
 
     # attention-kernel duration (events bracketing each attention launch)
     n_ev = min(args.steps, 200)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n_ev)]
     for i in range(n_ev):
         step(i, evs[i])
     torch.cuda.synchronize()
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
 
     flops = cnt["attn_flops"]
     value = world * flops / (step_ms * 1e-3) / 1e12
@@ -242,6 +248,14 @@ def run_ours(args, world, rank, local):
             "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 1.59 PF/s",
             "traffic": traffic,
             "attn_ms": round(attn_ms, 4),
+        },
+        "hbm_kernels": {
+            "pool_kv": {"ms": round(pool_ms, 4), "bytes": cnt["pool_bytes"],
+                        "GB/s": round(cnt["pool_bytes"] / (pool_ms * 1e-3) / 1e9, 1) if cnt["pool_bytes"] else None,
+                        "frac_of_measured_hbm": round(cnt["pool_bytes"] / (pool_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if cnt["pool_bytes"] else None},
+            "route": {"ms": round(route_ms, 4), "bytes": cnt["route_bytes"],
+                      "GB/s": round(cnt["route_bytes"] / (route_ms * 1e-3) / 1e9, 1) if cnt["route_bytes"] else None,
+                      "frac_of_measured_hbm": round(cnt["route_bytes"] / (route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if cnt["route_bytes"] else None},
         },
         "clocks": clocks,
         "gpu_launches": args.steps * layer.launches_per_forward(),
@@ -297,7 +311,7 @@ def run_also(args, name):
     sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True,
                                 "steps": max(50, args.steps // 4)})
     r = run_ours(sub, 1, 0, int(os.environ.get("LOCAL_RANK", "0")))
-    return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "gpu_launches")}
+    return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "hbm_kernels", "gpu_launches")}
 
 
 # ----------------------------------------------------------------- oracle (CPU)

@@ -12,6 +12,7 @@
 
 #include <cfloat>
 #include <climits>
+#include <algorithm>
 #include <mutex>
 
 #include "basa_internal.h"
@@ -19,8 +20,13 @@
 namespace basa {
 namespace {
 
-constexpr int kMeanThreads = 128;
-constexpr int kMeanUnroll = 4;
+__device__ __forceinline__ uint32_t ptx_pack(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+constexpr int kMeanThreads = 256;
 
 struct BoxMeanArgs {
   const void *src[2];
@@ -31,107 +37,129 @@ struct BoxMeanArgs {
   int bt, by, bx;     // box extents
   int nbt, nby, nbx;  // boxes per axis
   int ot, oy, ox;     // origin offset of box (0,0,0)
-  int nbox;
+  int nb_cta;         // boxes along x handled by one CTA
+  int splits;         // row splits per box (threads per (box, chunk))
+  int xgroups;        // CTAs along x = ceil(nbx / nb_cta)
   float inv_count;
 };
 
 __device__ __forceinline__ void accumulate(float *acc, const uint4 &v, const __nv_bfloat16 *) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __bfloat1622float2(h[e]);
-    acc[2 * e] += f.x;
-    acc[2 * e + 1] += f.y;
-  }
+  // bf16 -> fp32 is a 16-bit shift of the bit pattern
+  acc[0] += __uint_as_float(v.x << 16); acc[1] += __uint_as_float(v.x & 0xFFFF0000u);
+  acc[2] += __uint_as_float(v.y << 16); acc[3] += __uint_as_float(v.y & 0xFFFF0000u);
+  acc[4] += __uint_as_float(v.z << 16); acc[5] += __uint_as_float(v.z & 0xFFFF0000u);
+  acc[6] += __uint_as_float(v.w << 16); acc[7] += __uint_as_float(v.w & 0xFFFF0000u);
 }
 __device__ __forceinline__ void accumulate(float *acc, const uint4 &v, const float *) {
-  const float *f = reinterpret_cast<const float *>(&v);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) acc[e] += f[e];
+  acc[0] += __uint_as_float(v.x);
+  acc[1] += __uint_as_float(v.y);
+  acc[2] += __uint_as_float(v.z);
+  acc[3] += __uint_as_float(v.w);
 }
-__device__ __forceinline__ void store_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
-__device__ __forceinline__ void store_out(float *p, float x) { *p = x; }
+// Store the VEC means of one 16-byte input column: bfloat16 output (VEC = 8) or
+// float32 output (VEC = 8 from bfloat16 input, VEC = 4 from float32 input).
+template <int VEC>
+__device__ __forceinline__ void store_chunk(__nv_bfloat16 *p, const float *v) {
+  static_assert(VEC == 8, "bfloat16 output comes from bfloat16 input");
+  uint4 o;
+  o.x = ptx_pack(v[0], v[1]); o.y = ptx_pack(v[2], v[3]); o.z = ptx_pack(v[4], v[5]); o.w = ptx_pack(v[6], v[7]);
+  *reinterpret_cast<uint4 *>(p) = o;
+}
+template <int VEC>
+__device__ __forceinline__ void store_chunk(float *p, const float *v) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  if (VEC == 8) *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
 
-// One CTA per (tensor, b*head, box). A box is walked as rows of bx tokens (one
-// row per (t, y)); the row's bx * d elements are cut into 16-byte chunks and the
-// CTA's threads take consecutive chunks, so a warp reads contiguous bytes. A
-// thread always lands on the same chunk column c (128 is a multiple of the
-// chunks per token), keeps float32 sums for it, and the row/column position is
-// advanced incrementally (no division per load). Partial sums of the threads
-// that share a chunk column are reduced in shared memory at the end.
+// One CTA per (tensor, b*head, box row (t, y), group of nb_cta boxes along x).
+// Thread = (row split s, box i, 16-byte column c of the head dimension): it walks
+// rows s, s + splits, ... of its box and the box's x-run in each row with 32-bit
+// offsets (a box that wraps around the grid edge is two runs), keeping float32
+// sums of its 16 bytes. Adjacent threads read adjacent 16-byte columns, so a warp
+// reads whole contiguous token rows. Row splits are summed in shared memory.
 template <typename T, typename OutT>
-__global__ void __launch_bounds__(kMeanThreads) box_mean_kernel(BoxMeanArgs a) {
+__global__ void __launch_bounds__(kMeanThreads, 2) box_mean_kernel(BoxMeanArgs a) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ float red[];
   const int tensor = blockIdx.z;
-  const int bh = blockIdx.x / a.nbox;
-  const int box = blockIdx.x % a.nbox;
-  const int lpr = a.d / VEC;                 // chunks per token (8, 16 or 32)
-  const int chunk = threadIdx.x % lpr;       // fixed chunk column of this thread
-  const int slot = threadIdx.x / lpr;
-  const int jx = box % a.nbx, jy = (box / a.nbx) % a.nby, jt = box / (a.nbx * a.nby);
-  const int ot = (jt * a.bt + a.ot) % a.T, oy = (jy * a.by + a.oy) % a.H, ox = (jx * a.bx + a.ox) % a.W;
+  const int lpr = a.d / VEC;  // 16-byte columns per token
+  int rest = blockIdx.x;
+  const int xg = rest % a.xgroups; rest /= a.xgroups;
+  const int jy = rest % a.nby; rest /= a.nby;
+  const int jt = rest % a.nbt;
+  const int bh = rest / a.nbt;
+  const int c = threadIdx.x % lpr;
+  const int bi = (threadIdx.x / lpr) % a.nb_cta;
+  const int sp = threadIdx.x / (lpr * a.nb_cta);
+  const int jx = xg * a.nb_cta + bi;
+  const bool valid = jx < a.nbx && sp < a.splits;
   // select with conditionals: a dynamic index into the parameter arrays would copy them to local memory
   const void *src = tensor ? a.src[1] : a.src[0];
   const long long stride = tensor ? a.src_bh_stride[1] : a.src_bh_stride[0];
   void *dst = tensor ? a.dst[1] : a.dst[0];
-  const T *base = static_cast<const T *>(src) + (long long)bh * stride + chunk * VEC;
-  const int row_chunks = a.bx * lpr;
-  const int nrows = a.bt * a.by;
-  const int step_rows = kMeanThreads / row_chunks;  // whole rows advanced per step of 128 chunks
-  const int step_rem = kMeanThreads % row_chunks;
-  const int lpr_shift = __ffs(lpr) - 1;
-
-  // position of chunk index threadIdx.x: row r = (rt, ry), chunk xc within the row
-  int r = threadIdx.x / row_chunks, xc = threadIdx.x % row_chunks;
-  int rt = r / a.by, ry = r % a.by;
+  const uint4 *base = reinterpret_cast<const uint4 *>(static_cast<const T *>(src) + (long long)bh * stride) + c;
   float acc[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  auto advance = [&]() {
-    xc += step_rem;
-    int dr = step_rows;
-    if (xc >= row_chunks) { xc -= row_chunks; ++dr; }
-    r += dr;
-    ry += dr;
-    while (ry >= a.by) { ry -= a.by; ++rt; }
-  };
-  while (r < nrows) {
-    uint4 v[kMeanUnroll];
-#pragma unroll
-    for (int i = 0; i < kMeanUnroll; ++i) {
-      if (r < nrows) {
-        int t = ot + rt; t -= (t >= a.T) ? a.T : 0;
-        int y = oy + ry; y -= (y >= a.H) ? a.H : 0;
-        int x = ox + (xc >> lpr_shift); x -= (x >= a.W) ? a.W : 0;
-        const long long tok = ((long long)t * a.H + y) * a.W + x;
-        v[i] = __ldg(reinterpret_cast<const uint4 *>(base + tok * a.d));
-        advance();
-      } else {
-        v[i] = make_uint4(0, 0, 0, 0);
+  if (valid) {
+    const int ot = (jt * a.bt + a.ot) % a.T, oy = (jy * a.by + a.oy) % a.H, ox = (jx * a.bx + a.ox) % a.W;
+    const int run0 = min(a.bx, a.W - ox);  // tokens before the grid edge; the rest start at x = 0
+    const int nrows = a.bt * a.by;
+    int rt = sp / a.by, ry = sp % a.by;
+    for (int r = sp; r < nrows; r += a.splits) {
+      int t = ot + rt; t -= (t >= a.T) ? a.T : 0;
+      int y = oy + ry; y -= (y >= a.H) ? a.H : 0;
+      const uint32_t row = uint32_t(t * a.H + y) * uint32_t(a.W);
+      const uint4 *p0 = base + (row + uint32_t(ox)) * uint32_t(lpr);
+      int xx = 0;
+      for (; xx + 4 <= run0; xx += 4) {
+        const uint4 v0 = __ldg(p0 + (xx + 0) * lpr), v1 = __ldg(p0 + (xx + 1) * lpr);
+        const uint4 v2 = __ldg(p0 + (xx + 2) * lpr), v3 = __ldg(p0 + (xx + 3) * lpr);
+        accumulate(acc, v0, static_cast<const T *>(nullptr));
+        accumulate(acc, v1, static_cast<const T *>(nullptr));
+        accumulate(acc, v2, static_cast<const T *>(nullptr));
+        accumulate(acc, v3, static_cast<const T *>(nullptr));
       }
+      for (; xx < run0; ++xx) accumulate(acc, __ldg(p0 + xx * lpr), static_cast<const T *>(nullptr));
+      const uint4 *p1 = base + row * uint32_t(lpr);  // wrapped part of the run, from x = 0
+      for (int x1 = 0; x1 < a.bx - run0; ++x1) accumulate(acc, __ldg(p1 + x1 * lpr), static_cast<const T *>(nullptr));
+      ry += a.splits;
+      while (ry >= a.by) { ry -= a.by; ++rt; }
     }
-#pragma unroll
-    for (int i = 0; i < kMeanUnroll; ++i) accumulate(acc, v[i], static_cast<const T *>(nullptr));
   }
-  const int slots = kMeanThreads / lpr;
+  if (a.splits > 1) {
+    const int slot = threadIdx.x % (lpr * a.nb_cta);
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) red[slot * a.d + chunk * VEC + e] = acc[e];
-  __syncthreads();
-  for (int c = threadIdx.x; c < a.d; c += kMeanThreads) {
-    float s = 0.f;
-    for (int q = 0; q < slots; ++q) s += red[q * a.d + c];
-    OutT *out = static_cast<OutT *>(dst) + ((long long)bh * a.nbox + box) * a.d + c;
-    store_out(out, s * a.inv_count);
+    for (int e = 0; e < VEC; ++e) red[(sp * lpr * a.nb_cta + slot) * VEC + e] = acc[e];
+    __syncthreads();
+    if (sp == 0 && valid)
+      for (int q = 1; q < a.splits; ++q)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += red[(q * lpr * a.nb_cta + slot) * VEC + e];
+  }
+  if (sp == 0 && valid) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] *= a.inv_count;
+    const long long box = ((long long)jt * a.nby + jy) * a.nbx + jx;
+    const long long nbox = (long long)a.nbt * a.nby * a.nbx;
+    OutT *out = static_cast<OutT *>(dst) + ((long long)bh * nbox + box) * a.d + c * VEC;
+    store_chunk<VEC>(out, acc);
   }
 }
 
 template <typename T, typename OutT>
-basa_status run_box_mean(const BoxMeanArgs &a, int bh, cudaStream_t s) {
+basa_status run_box_mean(BoxMeanArgs a, int bh, cudaStream_t s) {
   const int lpr = a.d / (16 / int(sizeof(T)));
-  const size_t smem = size_t(kMeanThreads / lpr) * a.d * sizeof(float);
-  dim3 grid(unsigned(bh) * unsigned(a.nbox), 1, 2);
-  box_mean_kernel<T, OutT><<<grid, kMeanThreads, smem, s>>>(a);
+  a.nb_cta = std::max(1, std::min(a.nbx, kMeanThreads / lpr));
+  a.splits = std::max(1, kMeanThreads / (lpr * a.nb_cta));
+  a.splits = std::min(a.splits, a.bt * a.by);
+  a.xgroups = (a.nbx + a.nb_cta - 1) / a.nb_cta;
+  const int threads = lpr * a.nb_cta * a.splits;
+  const size_t smem = a.splits > 1 ? size_t(threads) * (16 / sizeof(T)) * sizeof(float) : 0;
+  const long long blocks = (long long)bh * a.nbt * a.nby * a.xgroups;
+  if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
+  dim3 grid(unsigned(blocks), 1, 2);
+  box_mean_kernel<T, OutT><<<grid, threads, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -218,7 +246,6 @@ basa_status launch_pool_kv(const void *k, const void *v, void *kp, void *vp, con
   a.bt = p.pt; a.by = p.ph; a.bx = p.pw;
   a.nbt = p.T / p.pt; a.nby = p.H / p.ph; a.nbx = p.W / p.pw;
   a.ot = a.oy = a.ox = 0;
-  a.nbox = a.nbt * a.nby * a.nbx;
   a.inv_count = 1.0f / float(p.pt * p.ph * p.pw);
   const int bh = p.B * p.heads;
   if (p.dtype == BASA_BF16) return run_box_mean<__nv_bfloat16, __nv_bfloat16>(a, bh, s);
@@ -241,7 +268,6 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
   a.bt = p.wt; a.by = p.wh; a.bx = p.ww;
   a.nbt = g.nWt; a.nby = g.nWy; a.nbx = g.nWx;
   a.ot = p.st; a.oy = p.sy; a.ox = p.sx;
-  a.nbox = g.nWin;
   a.inv_count = 1.0f / float(p.wt * p.wh * p.ww);
   basa_status st = (p.dtype == BASA_BF16) ? run_box_mean<__nv_bfloat16, float>(a, bh, s) : run_box_mean<float, float>(a, bh, s);
   if (st != BASA_OK) return st;
