@@ -122,7 +122,17 @@ __global__ void __launch_bounds__(kMeanThreads, 2) box_mean_kernel(BoxMeanArgs a
       }
       for (; xx < run0; ++xx) accumulate(acc, __ldg(p0 + xx * lpr), static_cast<const T *>(nullptr));
       const uint4 *p1 = base + row * uint32_t(lpr);  // wrapped part of the run, from x = 0
-      for (int x1 = 0; x1 < a.bx - run0; ++x1) accumulate(acc, __ldg(p1 + x1 * lpr), static_cast<const T *>(nullptr));
+      const int run1 = a.bx - run0;
+      int x1 = 0;
+      for (; x1 + 4 <= run1; x1 += 4) {
+        const uint4 v0 = __ldg(p1 + (x1 + 0) * lpr), v1 = __ldg(p1 + (x1 + 1) * lpr);
+        const uint4 v2 = __ldg(p1 + (x1 + 2) * lpr), v3 = __ldg(p1 + (x1 + 3) * lpr);
+        accumulate(acc, v0, static_cast<const T *>(nullptr));
+        accumulate(acc, v1, static_cast<const T *>(nullptr));
+        accumulate(acc, v2, static_cast<const T *>(nullptr));
+        accumulate(acc, v3, static_cast<const T *>(nullptr));
+      }
+      for (; x1 < run1; ++x1) accumulate(acc, __ldg(p1 + x1 * lpr), static_cast<const T *>(nullptr));
       ry += a.splits;
       while (ry >= a.by) { ry -= a.by; ++rt; }
     }
@@ -175,8 +185,9 @@ struct RouteArgs {
 };
 
 // One CTA per (b*head, group of 8 query windows); one warp per query window.
-// Km is staged through shared memory in chunks of 128 windows (rows padded by
-// one float so the lanes of a warp hit distinct banks).
+// Km is staged through shared memory in chunks of 128 windows, one warp per row
+// with 16-byte loads; rows are padded to d + 4 floats so that the 16-byte reads
+// of 8 consecutive rows by a quarter warp hit distinct banks.
 __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs a) {
   extern __shared__ float sm[];
   const int ngroups = (a.nwin + kRouteWarps - 1) / kRouteWarps;
@@ -185,27 +196,35 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int w = group * kRouteWarps + warp;
   const bool valid = w < a.nwin;
-  const int ld = a.d + 1;
-  float *kchunk = sm;                                        // [128][d+1]
-  float *qrow = kchunk + kRouteChunk * ld + warp * a.d;      // [8][d]
+  const int ld = a.d + 4;
+  const int d4 = a.d / 4;  // float4 per row
+  float *kchunk = sm;                                         // [128][d+4]
+  float *qrow = kchunk + kRouteChunk * ld + warp * a.d;       // [8][d]
   float *scores = kchunk + kRouteChunk * ld + kRouteWarps * a.d + warp * a.nwin;  // [8][nwin]
-  const float *qm = a.qm + (long long)bh * a.nwin * a.d;
-  const float *km = a.km + (long long)bh * a.nwin * a.d;
+  const float4 *qm = reinterpret_cast<const float4 *>(a.qm + (long long)bh * a.nwin * a.d);
+  const float4 *km = reinterpret_cast<const float4 *>(a.km + (long long)bh * a.nwin * a.d);
   if (valid)
-    for (int c = lane; c < a.d; c += 32) qrow[c] = qm[(long long)w * a.d + c];
+    for (int c = lane; c < d4; c += 32) reinterpret_cast<float4 *>(qrow)[c] = qm[(long long)w * d4 + c];
   for (int c0 = 0; c0 < a.nwin; c0 += kRouteChunk) {
     const int rows = min(kRouteChunk, a.nwin - c0);
     __syncthreads();
-    for (int i = threadIdx.x; i < rows * a.d; i += blockDim.x) {
-      const int r = i / a.d, c = i % a.d;
-      kchunk[r * ld + c] = km[(long long)(c0 + r) * a.d + c];
-    }
+    for (int r = warp; r < rows; r += kRouteWarps)
+      for (int c = lane; c < d4; c += 32)
+        reinterpret_cast<float4 *>(kchunk + r * ld)[c] = km[(long long)(c0 + r) * d4 + c];
     __syncthreads();
     if (valid)
       for (int r = lane; r < rows; r += 32) {
-        float s = 0.f;
-        for (int c = 0; c < a.d; ++c) s = fmaf(qrow[c], kchunk[r * ld + c], s);
-        scores[c0 + r] = (c0 + r == w) ? -INFINITY : s;
+        const float4 *kr = reinterpret_cast<const float4 *>(kchunk + r * ld);
+        const float4 *qr = reinterpret_cast<const float4 *>(qrow);
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int c = 0; c < d4; ++c) {
+          const float4 kv = kr[c], qv = qr[c];
+          s0 = fmaf(qv.x, kv.x, s0);
+          s1 = fmaf(qv.y, kv.y, s1);
+          s2 = fmaf(qv.z, kv.z, s2);
+          s3 = fmaf(qv.w, kv.w, s3);
+        }
+        scores[c0 + r] = (c0 + r == w) ? -INFINITY : (s0 + s1) + (s2 + s3);
       }
   }
   __syncwarp();
@@ -272,7 +291,7 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
   basa_status st = (p.dtype == BASA_BF16) ? run_box_mean<__nv_bfloat16, float>(a, bh, s) : run_box_mean<float, float>(a, bh, s);
   if (st != BASA_OK) return st;
   RouteArgs r{qm, km, route_idx, route_score, g.nWin, p.head_dim, p.routed_k};
-  const size_t smem = (size_t(kRouteChunk) * (p.head_dim + 1) + kRouteWarps * p.head_dim + size_t(kRouteWarps) * g.nWin) * sizeof(float);
+  const size_t smem = (size_t(kRouteChunk) * (p.head_dim + 4) + kRouteWarps * p.head_dim + size_t(kRouteWarps) * g.nWin) * sizeof(float);
   static bool attr_set[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BASA_ERR_CUDA;
