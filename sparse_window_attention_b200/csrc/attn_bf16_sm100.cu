@@ -336,15 +336,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       c.wtype[1 + r] = t;
       c.org[1 + r][0] = a; c.org[1 + r][1] = b; c.org[1 + r][2] = d;
     }
-    // column masks of this CTA's key tiles, in stream order (all ones = full tile)
-    uint4 *tab = reinterpret_cast<uint4 *>(smem + kSmemMask);
-    KeyIter it{0, 0};
-    for (int j = 0; j < kMaskTable && it.seg <= P.routed_k + 2; ++j) {
-      uint32_t m[4];
-      key_tile_mask(P, c, it, m);
-      tab[j] = make_uint4(m[0], m[1], m[2], m[3]);
-      advance(P, c, it);
-    }
     ptx::fence_mbar_init();
   }
   if (P.plan.zero_fill) {
@@ -373,12 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     if (lane == 0) {
       Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, true};
       Waiter drain{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
-      uint32_t qbytes = 0;
-      for (int g = 0; g < (has_q1 ? 2 : 1); ++g) {
-        const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
-        for (int i = 0; i < tile.n_pieces; ++i)
-          qbytes += uint32_t(P.plan.shape[P.plan.piece[tile.first_piece + i].shape].rows) * 256u;
-      }
+      // a tile's TMA boxes deliver 256 bytes per valid row (two 128-byte halves)
+      uint32_t qbytes = uint32_t(P.plan.tile[ty.first_tile + q_tile0].valid_rows) * 256u;
+      if (has_q1) qbytes += uint32_t(P.plan.tile[ty.first_tile + q_tile0 + 1].valid_rows) * 256u;
       ptx::mbar_arrive_expect_tx(&c.q_full, qbytes);
       for (int g = 0; g < (has_q1 ? 2 : 1); ++g)
         load_window_tile(P, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh, smem + kSmemQ + g * kTileBytes,
@@ -395,14 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
           if (item == 0 && (P.flags & BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD)) { skipped0 = true; last = item; continue; }
           uint8_t *dst = smem + kSmemRing + slot * kTileBytes;
           // Arm the barrier with the byte count before issuing the copies.
-          uint32_t bytes = 0;
-          if (it.seg <= P.routed_k) {
-            const PlanTile &tile = P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t];
-            for (int i = 0; i < tile.n_pieces; ++i)
-              bytes += uint32_t(P.plan.shape[P.plan.piece[tile.first_piece + i].shape].rows) * 256u;
-          } else {
-            bytes = kTileBytes;
-          }
+          const uint32_t bytes = it.seg <= P.routed_k
+                                     ? uint32_t(P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t].valid_rows) * 256u
+                                     : kTileBytes;
           ptx::mbar_arrive_expect_tx(&c.full[slot], bytes);
           load_key_tile(P, c, it, kv == 1, bh, dst, &c.full[slot]);
           last = item;
@@ -489,6 +472,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     uint8_t *q_tile = smem + kSmemQ + g * kTileBytes;
     const uint32_t swz = row & 7;
     const float sl2 = P.scale_log2;
+    {
+      // Column masks of this CTA's key tiles in stream order (all ones = full tile),
+      // one tile per softmax thread; this runs while the first loads are in flight.
+      const int j = threadIdx.x - 64;
+      if (j < kMaskTable && j < n_kt) {
+        KeyIter t{0, j};
+        while (t.seg <= P.routed_k + 2 && t.t >= seg_tiles(P, c, t.seg)) {
+          t.t -= seg_tiles(P, c, t.seg);
+          ++t.seg;
+        }
+        uint32_t mk[4];
+        key_tile_mask(P, c, t, mk);
+        reinterpret_cast<uint4 *>(smem + kSmemMask)[j] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
+      }
+      ptx::named_barrier(3, 256);  // the 256 softmax threads
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = active;
     KeyIter it{0, 0};
