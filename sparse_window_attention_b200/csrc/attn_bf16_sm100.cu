@@ -66,6 +66,7 @@ struct alignas(64) AttnParams {
   Geo g;
   int routed_k, n_pool, n_text, n_pool_tiles, n_text_tiles;
   float scale_log2;
+  int all_full;  // every key tile of the launch is full: no column masks
   uint32_t flags;
   unsigned long long timeout_ns;
 };
@@ -498,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       uint32_t s[128];
       ptx::tmem_ld128(tS, s);
       ptx::tmem_ld_wait(s);
-      if (j < kMaskTable) {
+      if (P.all_full) {
+      } else if (j < kMaskTable) {
         const uint4 mt = reinterpret_cast<const uint4 *>(smem + kSmemMask)[j];
         if ((mt.x & mt.y & mt.z & mt.w) != 0xFFFFFFFFu) {
           const uint32_t mask[4] = {mt.x, mt.y, mt.z, mt.w};
@@ -675,6 +677,8 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
   P.routed_k = p.routed_k;
   P.scale_log2 = float(1.4426950408889634 / std::sqrt(double(p.head_dim)));
   P.flags = p.flags;
+  P.all_full = (P.n_pool % kTileRows == 0) && (p.n_text % kTileRows == 0);
+  for (int i = 0; i < P.plan.n_tiles; ++i) P.all_full &= P.plan.tile[i].valid_rows == kTileRows;
   P.timeout_ns = (p.wait_timeout_us ? (unsigned long long)p.wait_timeout_us : 2000000ull) * 1000ull;
   const long long blocks = (long long)p.B * p.heads * P.g.nWin * P.plan.max_pairs;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;

@@ -208,9 +208,21 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs 
   for (int c0 = 0; c0 < a.nwin; c0 += kRouteChunk) {
     const int rows = min(kRouteChunk, a.nwin - c0);
     __syncthreads();
-    for (int r = warp; r < rows; r += kRouteWarps)
-      for (int c = lane; c < d4; c += 32)
-        reinterpret_cast<float4 *>(kchunk + r * ld)[c] = km[(long long)(c0 + r) * d4 + c];
+    // all loads of a thread first (independent), then the shared-memory stores
+    constexpr int kPer = kRouteChunk / kRouteWarps;  // rows per warp
+    for (int c = lane; c < d4; c += 32) {
+      float4 v[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int r = warp + i * kRouteWarps;
+        if (r < rows) v[i] = km[(long long)(c0 + r) * d4 + c];
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int r = warp + i * kRouteWarps;
+        if (r < rows) reinterpret_cast<float4 *>(kchunk + r * ld)[c] = v[i];
+      }
+    }
     __syncthreads();
     if (valid)
       for (int r = lane; r < rows; r += 32) {
