@@ -154,7 +154,8 @@ def run_ours(args, world, rank, local):
     shifts = synth.SHIFT_CYCLES[args.workload]
     q, k, v = synth.make_inputs(wl, seed=args.seed + rank)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
-    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
+                      route_radius=wl.route_radius)
     out = torch.empty_like(qd)
     stream = torch.cuda.current_stream()
 
@@ -228,7 +229,8 @@ def run_ours(args, world, rank, local):
         "config": {
             "workload": f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} grid={'x'.join(map(str, wl.grid))} "
                         f"window={'x'.join(map(str, wl.window))} shifts={shifts} pool={'x'.join(map(str, wl.pool))} "
-                        f"text={wl.n_text} routed_k={wl.routed_k}",
+                        f"text={wl.n_text} routed_k={wl.routed_k}"
+                        + (f" route_radius={wl.route_radius}" if wl.route_radius else ""),
             "keys_per_query": cnt["keys_per_query"],
             "attn_gflop_per_layer": round(flops / 1e9, 2),
             "parallelism": f"(batch, head) units sharded over {world} GPU(s), {wl.B * wl.heads} per GPU, no data-path collective",
@@ -262,8 +264,10 @@ def run_ours(args, world, rank, local):
     }
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world)
-    if not args.no_extra and world == 1 and args.workload != "wan":
-        res["also_wan"] = run_also(args, "wan")
+    if not args.no_extra and world == 1:
+        for name in ("wan", "wan_video"):
+            if args.workload != name:
+                res["also_" + name] = run_also(args, name)
     return res
 
 
@@ -308,8 +312,9 @@ def run_e2e(args, layer, q, k, v, shifts, flops, world):
 
 def run_also(args, name):
     """Secondary workload on the same GPU (context for the headline line)."""
-    sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True,
-                                "steps": max(50, args.steps // 4)})
+    # about a second of timed work each: a video layer is ~50x a FLUX-2K layer
+    steps = max(10, args.steps // 50) if name == "wan_video" else max(50, args.steps // 4)
+    sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True, "steps": steps})
     r = run_ours(sub, 1, 0, int(os.environ.get("LOCAL_RANK", "0")))
     return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "hbm_kernels", "gpu_launches")}
 

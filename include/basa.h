@@ -87,6 +87,11 @@ typedef struct {
   uint32_t flags;          /* 0, or BASA_FLAG_TEST_* hooks                              */
   uint32_t wait_timeout_us;/* limit of each bounded wait inside the attention kernel;
                               0 = default (2,000,000 us)                               */
+  int route_radius;        /* routing candidates: 0 = every other window; r >= 1 = the
+                              windows whose window-grid index differs from the query
+                              window's by at most r along each axis (no wrap-around).
+                              routed_k must not exceed the fewest candidates any window
+                              has: prod over axes of (min(r, nW_axis - 1) + 1), minus 1 */
 } basa_params;
 
 /*
@@ -116,8 +121,13 @@ size_t basa_route_workspace_bytes(const basa_params *p);
  *
  *   Qm[w] = mean of q over the tokens of shifted window w     (float32)
  *   Km[u] = mean of k over the tokens of shifted window u     (float32)
- *   score[w,u] = Qm[w] . Km[u]  for u != w
- *   route_idx[b,h,w,:] = the routed_k windows u with the largest scores,
+ *   score[w,u] = Qm[w] . Km[u]  for candidates u of w: every u != w, or with
+ *                route_radius = r >= 1 only those u != w whose window-grid
+ *                coordinates (jt, jy, jx) differ from w's by at most r on every
+ *                axis, counted without wrap-around (BASA §A.2: one routed window
+ *                per query window, candidate-window radius one, in the video
+ *                configuration)
+ *   route_idx[b,h,w,:] = the routed_k candidates u with the largest scores,
  *                        ties to the lower id, by descending score
  *   route_score[b,h,w,:] = their scores (optional: pass NULL to skip)
  * Requires routed_k >= 1. `workspace` is a device buffer of at least

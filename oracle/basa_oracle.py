@@ -23,12 +23,13 @@ blocking, fusion or reordering beyond what the definition needs:
    branches are equivalent to one softmax over concatenated K/V);
 6. inverse shift of the output.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * shift convention Xr[t,y,x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W] (roll by -s);
   * window ids are raster order over the window grid of the shifted frame;
   * routing score = dot product of float64 window means of Q and K, the window
-    itself excluded, candidates = all other windows, ties to the lower id, the
-    chosen ids listed by descending score;
+    itself excluded, candidates = all other windows or, with a radius r, the
+    windows within Chebyshev distance r on the window grid (no wrap-around),
+    ties to the lower id, the chosen ids listed by descending score;
   * text tokens are keys only (rows N.. of k and v); only visual queries are output;
   * pooled tokens are listed in raster order of the pooled grid.
 
@@ -52,6 +53,7 @@ class Geometry:
     pool: tuple = (0, 0, 0)  # (pt, ph, pw); all zero = no pooled keys
     n_text: int = 0
     routed_k: int = 0
+    route_radius: int = 0  # 0 = every other window is a routing candidate
 
     @property
     def N(self):
@@ -149,25 +151,57 @@ def window_means(q, k, geo: Geometry):
     return out[0], out[1]
 
 
+def window_coords(geo: Geometry, w: int):
+    """Window-grid coordinates (jt, jy, jx) of window id w (raster order)."""
+    nt, ny, nx = geo.win_grid
+    return w // (ny * nx), (w // nx) % ny, w % nx
+
+
+def candidate_windows(geo: Geometry, w: int):
+    """Windows that may be routed to query window w, in increasing id order.
+
+    Every other window when geo.route_radius == 0. With a radius r >= 1, the other
+    windows of the (2r+1)^3 block of the window grid centred on w, clipped at the
+    grid's edges (BASA §A.2: candidate-window radius one in the video configuration;
+    the distance is read as Chebyshev distance between window-grid coordinates,
+    without wrap-around).
+    """
+    r = geo.route_radius
+    nt, ny, nx = geo.win_grid
+    if r == 0:
+        return [u for u in range(geo.n_win) if u != w]
+    jt, jy, jx = window_coords(geo, w)
+    out = []
+    for ut in range(max(0, jt - r), min(nt, jt + r + 1)):
+        for uy in range(max(0, jy - r), min(ny, jy + r + 1)):
+            for ux in range(max(0, jx - r), min(nx, jx + r + 1)):
+                u = (ut * ny + uy) * nx + ux
+                if u != w:
+                    out.append(u)
+    return out
+
+
 def route_windows(q, k, geo: Geometry):
     """Top-k routed windows per query window (BASA §3.3, content-adaptive routing).
 
-    score[w, u] = mean(Q over window w) . mean(K over window u), u != w. The k
-    windows with the largest scores are kept, ties going to the lower window id,
-    listed by descending score. Returns (route_idx int32 [B,h,nWin,k],
-    scores float64 [B,h,nWin,nWin] with the diagonal set to -inf).
+    score[w, u] = mean(Q over window w) . mean(K over window u) for the candidates u
+    of w (candidate_windows). The k candidates with the largest scores are kept,
+    ties going to the lower window id, listed by descending score. Returns
+    (route_idx int32 [B,h,nWin,k], scores float64 [B,h,nWin,nWin] with every
+    non-candidate entry, the diagonal included, set to -inf).
     """
     Qm, Km = window_means(q, k, geo)
     S = np.einsum("bhwd,bhud->bhwu", Qm, Km)
     nw = geo.n_win
-    S[..., np.arange(nw), np.arange(nw)] = -np.inf
     B, h = S.shape[:2]
     idx = np.zeros((B, h, nw, geo.routed_k), dtype=np.int32)
-    ids = np.arange(nw)
-    for b in range(B):
-        for hh in range(h):
-            for w in range(nw):
-                cand = ids[ids != w]
+    for w in range(nw):
+        cand = np.array(candidate_windows(geo, w), dtype=np.int64)
+        keep = np.zeros(nw, dtype=bool)
+        keep[cand] = True
+        S[:, :, w, ~keep] = -np.inf
+        for b in range(B):
+            for hh in range(h):
                 sc = S[b, hh, w, cand]
                 order = np.lexsort((cand, -sc))  # primary: score descending, then id ascending
                 idx[b, hh, w] = cand[order[: geo.routed_k]]

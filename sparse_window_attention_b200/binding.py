@@ -54,6 +54,7 @@ class basa_params(ctypes.Structure):
         ("dev_err", ctypes.c_void_p),
         ("flags", ctypes.c_uint32),
         ("wait_timeout_us", ctypes.c_uint32),
+        ("route_radius", ctypes.c_int),
     ]
 
 
@@ -84,7 +85,7 @@ _lib = load_library()
 
 
 def make_params(B, heads, head_dim, grid, window, shift=(0, 0, 0), pool=(0, 0, 0), n_text=0, routed_k=0,
-                dtype="bf16", dev_err=None, flags=0, wait_timeout_us=0) -> basa_params:
+                dtype="bf16", dev_err=None, flags=0, wait_timeout_us=0, route_radius=0) -> basa_params:
     p = basa_params()
     p.B, p.heads, p.head_dim = B, heads, head_dim
     p.T, p.H, p.W = grid
@@ -96,6 +97,7 @@ def make_params(B, heads, head_dim, grid, window, shift=(0, 0, 0), pool=(0, 0, 0
     p.dev_err = _ptr(dev_err)
     p.flags = flags
     p.wait_timeout_us = wait_timeout_us
+    p.route_radius = route_radius
     return p
 
 

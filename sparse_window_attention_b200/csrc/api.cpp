@@ -13,6 +13,15 @@ bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 bool empty_batch(const basa_params *p) { return p->B == 0 || p->heads == 0; }
 
+// Fewest routing candidates of any window under a radius r >= 1: a corner window
+// sees min(r, n - 1) + 1 window positions along an axis of n windows.
+int64_t min_candidates(const basa_params *p) {
+  const int64_t n[3] = {p->T / p->wt, p->H / p->wh, p->W / p->ww};
+  int64_t c = 1;
+  for (int a = 0; a < 3; ++a) c *= (n[a] - 1 < p->route_radius ? n[a] - 1 : p->route_radius) + 1;
+  return c - 1;
+}
+
 // Checks shared by every entry point.
 basa_status check_common(const basa_params *p) {
   if (!p) return BASA_ERR_INVALID_ARG;
@@ -34,8 +43,10 @@ basa_status check_common(const basa_params *p) {
   const int64_t bh = int64_t(p->B) * p->heads;
   if (bh >= (int64_t(1) << 31)) return BASA_ERR_UNSUPPORTED;
   const int64_t nwin = N / (int64_t(p->wt) * p->wh * p->ww);
+  if (p->route_radius < 0) return BASA_ERR_INVALID_ARG;
   if (p->routed_k > 0) {
     if (p->routed_k > basa::kMaxRouted || p->routed_k > nwin - 1) return BASA_ERR_INVALID_ARG;
+    if (p->route_radius > 0 && p->routed_k > min_candidates(p)) return BASA_ERR_INVALID_ARG;
   }
   return BASA_OK;
 }

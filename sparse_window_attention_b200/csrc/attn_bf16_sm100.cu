@@ -71,6 +71,9 @@ struct alignas(64) AttnParams {
   unsigned long long timeout_ns;
 };
 
+// __grid_constant__ kernel parameters are limited to 32764 bytes.
+static_assert(sizeof(AttnParams) <= 32764, "window plan too large for the kernel parameter space");
+
 struct Ctrl {
   uint64_t full[kStages], empty[kStages];
   uint64_t q_full, s_full[2], p_full[2], o_full[2], drain;

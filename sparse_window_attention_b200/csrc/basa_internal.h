@@ -27,8 +27,8 @@ namespace basa {
 // ---------------------------------------------------------------------------
 constexpr int kTileRows = 128;
 constexpr int kMaxShapes = 8;
-constexpr int kMaxPieces = 256;
-constexpr int kMaxTiles = 128;
+constexpr int kMaxPieces = 1024;
+constexpr int kMaxTiles = 512;
 constexpr int kMaxRouted = 16;
 
 struct PlanShape {

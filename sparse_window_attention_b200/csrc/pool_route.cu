@@ -5,9 +5,10 @@
 //    global memory over the UNSHIFTED grid); with box = window and offset = shift
 //    (boxes wrap around the grid edge) it gives the window means of Q and K used
 //    by the routing of BASA §3.3.
-//  * route_topk_kernel: score[w,u] = Qm[w] . Km[u] (u != w) and a warp-level top-k
+//  * route_topk_kernel: score[w,u] = Qm[w] . Km[u] over the candidates u of w (every
+//    u != w, or the windows within a window-grid radius) and a warp-level top-k
 //    per query window, ties to the lower window id (BASA §3.3 content-adaptive
-//    true-window routing).
+//    true-window routing; §A.2 candidate-window radius).
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -182,7 +183,19 @@ struct RouteArgs {
   int32_t *idx;
   float *score;
   int nwin, d, k;
+  int radius;           // 0 = every other window is a candidate
+  int nwy, nwx;         // window grid extents along y and x
 };
+
+// Window u is a routing candidate of window w: u != w and, under a radius r >= 1,
+// their window-grid coordinates differ by at most r on every axis (no wrap-around).
+__device__ __forceinline__ bool route_candidate(const RouteArgs &a, int w, int u) {
+  if (u == w) return false;
+  if (a.radius == 0) return true;
+  const int wx = w % a.nwx, wy = (w / a.nwx) % a.nwy, wt = w / (a.nwx * a.nwy);
+  const int ux = u % a.nwx, uy = (u / a.nwx) % a.nwy, ut = u / (a.nwx * a.nwy);
+  return abs(wx - ux) <= a.radius && abs(wy - uy) <= a.radius && abs(wt - ut) <= a.radius;
+}
 
 // One CTA per (b*head, group of 8 query windows); one warp per query window.
 // Km is staged through shared memory in chunks of 128 windows, one warp per row
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs 
           s2 = fmaf(qv.z, kv.z, s2);
           s3 = fmaf(qv.w, kv.w, s3);
         }
-        scores[c0 + r] = (c0 + r == w) ? -INFINITY : (s0 + s1) + (s2 + s3);
+        scores[c0 + r] = route_candidate(a, w, c0 + r) ? (s0 + s1) + (s2 + s3) : -INFINITY;
       }
   }
   __syncwarp();
@@ -302,7 +315,7 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
   a.inv_count = 1.0f / float(p.wt * p.wh * p.ww);
   basa_status st = (p.dtype == BASA_BF16) ? run_box_mean<__nv_bfloat16, float>(a, bh, s) : run_box_mean<float, float>(a, bh, s);
   if (st != BASA_OK) return st;
-  RouteArgs r{qm, km, route_idx, route_score, g.nWin, p.head_dim, p.routed_k};
+  RouteArgs r{qm, km, route_idx, route_score, g.nWin, p.head_dim, p.routed_k, p.route_radius, g.nWy, g.nWx};
   const size_t smem = (size_t(kRouteChunk) * (p.head_dim + 4) + kRouteWarps * p.head_dim + size_t(kRouteWarps) * g.nWin) * sizeof(float);
   static bool attr_set[64] = {false};
   int dev = 0;

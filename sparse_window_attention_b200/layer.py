@@ -14,10 +14,11 @@ from . import binding as B
 
 class BasaLayer:
     def __init__(self, batch, heads, head_dim, grid, window, pool=(0, 0, 0), n_text=0, routed_k=0, dtype="bf16",
-                 device="cuda"):
+                 device="cuda", route_radius=0):
         self.batch, self.heads, self.head_dim = batch, heads, head_dim
         self.grid, self.window, self.pool = tuple(grid), tuple(window), tuple(pool)
         self.n_text, self.routed_k, self.dtype = n_text, routed_k, dtype
+        self.route_radius = route_radius
         self.device = torch.device(device)
         T, H, W = self.grid
         self.N = T * H * W
@@ -43,7 +44,7 @@ class BasaLayer:
         if key not in self._params:
             self._params[key] = B.make_params(self.batch, self.heads, self.head_dim, self.grid, self.window, shift,
                                               self.pool, self.n_text, self.routed_k, self.dtype,
-                                              dev_err=self.dev_err, **extra)
+                                              dev_err=self.dev_err, route_radius=self.route_radius, **extra)
         return self._params[key]
 
     def pool_kv(self, k, v, shift=(0, 0, 0), stream=None):

@@ -91,6 +91,7 @@ class Workload:
     n_text: int
     routed_k: int
     field: str  # "iid", "sinusoid" or "block_mean"
+    route_radius: int = 0  # routing candidates: 0 = all other windows, r = window-grid radius r
 
     @property
     def N(self) -> int:
@@ -101,13 +102,19 @@ class Workload:
         return Workload(**{**self.__dict__, "shift": tuple(shift)})
 
 
-# The five workload shapes (B=1). Shift cycles are listed in SHIFT_CYCLES.
+# Workload shapes (B=1). Shift cycles are listed in SHIFT_CYCLES.
 WORKLOADS = {
     "tiny": Workload("tiny", "f32", 1, 2, 64, (1, 32, 32), (1, 8, 8), (0, 4, 4), (1, 4, 4), 0, 0, "iid"),
     "flux1k": Workload("flux1k", "bf16", 1, 24, 128, (1, 64, 64), (1, 16, 16), (0, 0, 0), (1, 8, 8), 512, 0, "sinusoid"),
     "flux2k": Workload("flux2k", "bf16", 1, 24, 128, (1, 128, 128), (1, 32, 32), (0, 0, 0), (1, 8, 8), 512, 0, "sinusoid"),
     "flux4k": Workload("flux4k", "bf16", 1, 24, 128, (1, 256, 256), (1, 32, 32), (0, 16, 16), (1, 16, 16), 512, 0, "sinusoid"),
     "wan": Workload("wan", "bf16", 1, 12, 128, (21, 30, 52), (3, 6, 13), (0, 3, 6), (3, 6, 13), 0, 4, "block_mean"),
+    # The pages' own video configuration at the Wan2.1-1.3B latent grid of 1664x960, 81
+    # frames: windows keep the full temporal extent, pooling is spatial only, and one
+    # routed window is chosen among the radius-one neighbours (BASA §3.2, §3.3, §A.2 and
+    # Table 3, row w=(15,26), p=(4,4)).
+    "wan_video": Workload("wan_video", "bf16", 1, 12, 128, (21, 60, 104), (21, 15, 26), (0, 7, 13), (1, 4, 4), 0, 1,
+                          "block_mean", route_radius=1),
 }
 
 SHIFT_CYCLES = {
@@ -116,6 +123,7 @@ SHIFT_CYCLES = {
     "flux2k": [(0, 0, 0), (0, 16, 0), (0, 0, 16), (0, 16, 16)],
     "flux4k": [(0, 16, 16)],
     "wan": [(0, 3, 6)],
+    "wan_video": [(0, 0, 0), (0, 7, 13)],
 }
 
 

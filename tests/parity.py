@@ -16,7 +16,7 @@ ROUTE_SCORE_TOL = 1e-3
 
 def geometry(wl, shift=None) -> O.Geometry:
     return O.Geometry(grid=wl.grid, window=wl.window, shift=tuple(shift if shift is not None else wl.shift),
-                      pool=wl.pool, n_text=wl.n_text, routed_k=wl.routed_k)
+                      pool=wl.pool, n_text=wl.n_text, routed_k=wl.routed_k, route_radius=wl.route_radius)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:

@@ -33,17 +33,18 @@ def test_status_strings():
 
 
 def test_params_struct_layout_matches_header():
-    # 18 ints, a pointer, two uint32 -> 72 + 8 + 8 bytes on LP64
-    assert ctypes.sizeof(B.basa_params) == 88
+    # 18 ints, a pointer, two uint32, an int -> 72 + 8 + 8 + 4 (+4 padding) bytes on LP64
+    assert ctypes.sizeof(B.basa_params) == 96
     assert B.basa_params.dev_err.offset == 72
+    assert B.basa_params.route_radius.offset == 88
 
 
 def _p(**kw):
     base = dict(B=1, heads=2, head_dim=128, grid=(1, 64, 64), window=(1, 16, 16), shift=(0, 8, 8), pool=(1, 8, 8),
-                n_text=16, routed_k=0, dtype="bf16")
+                n_text=16, routed_k=0, dtype="bf16", route_radius=0)
     base.update(kw)
     return B.make_params(base["B"], base["heads"], base["head_dim"], base["grid"], base["window"], base["shift"],
-                         base["pool"], base["n_text"], base["routed_k"], base["dtype"])
+                         base["pool"], base["n_text"], base["routed_k"], base["dtype"], route_radius=base["route_radius"])
 
 
 FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every case fails its checks first
@@ -64,6 +65,10 @@ FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every case fails i
         (dict(routed_k=17, grid=(1, 128, 128)), 1),
         (dict(B=-1), 1),
         (dict(dtype=7), 1),
+        (dict(route_radius=-1), 1),
+        # a corner window of the 1x4x4 window grid has 3 neighbours within radius 1
+        (dict(routed_k=4, route_radius=1), 1),
+        (dict(routed_k=9, route_radius=2, grid=(1, 128, 128)), 1),
     ],
 )
 def test_invalid_params_rejected_before_launch(kw, status):
@@ -100,6 +105,18 @@ def test_empty_batch_is_a_no_op():
         p = _p(**kw)
         assert B.basa_window_attn_fwd(None, None, None, None, None, None, None, p, stream=0, check=False) == 0
         assert B.basa_pool_kv(None, None, None, None, p, stream=0, check=False) == 0
+
+
+def test_route_radius_limits_routed_k():
+    """routed_k may reach the fewest candidates any window has under the radius."""
+    assert B.basa_route_workspace_bytes(_p(routed_k=3, route_radius=1)) > 0
+    assert B.basa_route_workspace_bytes(_p(routed_k=4, route_radius=1)) == 0
+    # 8x8 window grid, radius 2: a corner sees 3 x 3 positions, itself included
+    assert B.basa_route_workspace_bytes(_p(routed_k=8, route_radius=2, grid=(1, 128, 128))) > 0
+    assert B.basa_route_workspace_bytes(_p(routed_k=9, route_radius=2, grid=(1, 128, 128))) == 0
+    # the full video configuration: 4x4 spatial window grid, one routed window
+    p = B.make_params(1, 12, 128, (21, 60, 104), (21, 15, 26), (0, 7, 13), (1, 4, 4), 0, 1, "bf16", route_radius=1)
+    assert B.basa_route_workspace_bytes(p) == 2 * 12 * 16 * 128 * 4
 
 
 def test_route_workspace_bytes():

@@ -24,7 +24,8 @@ W = synth.Workload
 def _layer(wl):
     from sparse_window_attention_b200.layer import BasaLayer
 
-    return BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    return BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
+                     route_radius=wl.route_radius)
 
 
 def _heads(wl):
@@ -114,6 +115,74 @@ def test_tiny_f32():
     run_parity(synth.WORKLOADS["tiny"], (0, 4, 4))
 
 
+def sampled_rows(geo, n_random, seed):
+    """Query tokens to check on a large grid: random ones plus the first and last
+    tokens (shifted-frame raster order) of every window, which sit in the first and
+    last, ragged, query tiles."""
+    rng = np.random.default_rng(seed)
+    win = O.window_of_token(geo)
+    picks = set(rng.choice(geo.N, size=n_random, replace=False).tolist())
+    for w in range(geo.n_win):
+        members = np.nonzero(win == w)[0]  # original indices; shifted order differs
+        picks.update(members[[0, len(members) // 2, -1]].tolist())
+    return np.array(sorted(picks))
+
+
+_LARGE = {}  # the last large workload's inputs, reused across its shifts
+
+
+def _large_inputs(wl, seed):
+    key = (wl.name, seed)
+    if key not in _LARGE:
+        _LARGE.clear()
+        (q, k, v), dev = PT.gpu_inputs(wl, seed)
+        hs = _heads(wl)
+        _LARGE[key] = (dev, (PT.to64(q[:, hs]), PT.to64(k[:, hs]), PT.to64(v[:, hs])))
+    return _LARGE[key]
+
+
+def run_sampled_parity(wl, shift, n_random=96, seed=0):
+    """Full-size pool and routing parity on a head subset, attention parity on
+    sampled query rows (the oracle computes them one by one)."""
+    (qd, kd, vd), (q64, k64, v64) = _large_inputs(wl, seed)
+    geo = PT.geometry(wl, shift)
+    hs = _heads(wl)
+    layer = _layer(wl)
+    layer.pool_kv(kd, vd, shift)
+    layer.route(qd, kd, shift)
+    torch.cuda.synchronize()
+    kp_ex, vp_ex = O.pool_kv(k64, v64, geo)
+    PT.assert_pool_close(PT.to64(layer.kp[:, hs]), kp_ex, wl.dtype)
+    PT.assert_pool_close(PT.to64(layer.vp[:, hs]), vp_ex, wl.dtype)
+    route_or, S = O.route_windows(q64, k64, geo)
+    differing = PT.check_routes(layer.route_idx[:, hs].cpu().numpy(), route_or, S)
+    kp_or, vp_or = PT.oracle_pool_for_gpu(k64, v64, geo, wl.dtype)
+    kp_dev, vp_dev, route_dev = layer.kp.clone(), layer.vp.clone(), layer.route_idx.clone()
+    kp_dev[:, hs] = PT.to_device(kp_or, wl.dtype)
+    vp_dev[:, hs] = PT.to_device(vp_or, wl.dtype)
+    route_dev[:, hs] = torch.from_numpy(route_or).to(route_dev.device)
+    out = torch.full_like(qd, float("nan"))
+    layer.attention(qd, kd, vd, out, shift, kp=kp_dev, vp=vp_dev, route_idx=route_dev)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    assert not torch.isnan(out).any()  # every query row was written
+    rows = sampled_rows(geo, n_random, seed)
+    for j in range(len(hs)):
+        ref = O.attention_rows(q64, k64, v64, geo, 0, j, rows, kp=kp_or, vp=vp_or, route_idx=route_or)
+        PT.assert_outputs_close(PT.to64(out[0, hs[j]][rows]), ref, wl.dtype, f"{wl.name} head {hs[j]}")
+    return differing
+
+
+@pytest.mark.parametrize("shift", synth.SHIFT_CYCLES["wan_video"])
+def test_wan_video_full_size(shift):
+    """The pages' video configuration at 21x60x104: 15x26 spatial windows over all
+    frames, spatial-only 4x4 pooling, one routed window among radius-one neighbours."""
+    differing = run_sampled_parity(synth.WORKLOADS["wan_video"], shift)
+    assert differing == 0
+    if shift == synth.SHIFT_CYCLES["wan_video"][-1]:
+        _LARGE.clear()
+
+
 # ----------------------------------------------------------------- small shapes, edge cases
 
 SMALL = [
@@ -132,6 +201,14 @@ SMALL = [
     # float32 variants: head_dim 128, routing, text
     W("f32_d128", "f32", 1, 2, 128, (2, 16, 16), (1, 8, 8), (1, 4, 2), (2, 4, 4), 9, 2, "block_mean"),
     W("f32_d64", "f32", 2, 3, 64, (1, 24, 16), (1, 8, 8), (0, 5, 3), (1, 4, 4), 0, 1, "iid"),
+    # video variant: windows over all frames, spatial-only pooling, radius-one routing
+    W("video", "bf16", 1, 2, 128, (5, 24, 32), (5, 6, 8), (0, 3, 4), (1, 2, 2), 0, 1, "block_mean", route_radius=1),
+    # the same with a temporal shift (every window wraps in t) and the most routed
+    # windows radius one allows on a 4x4 window grid (a corner has 3 neighbours)
+    W("video_tshift", "bf16", 1, 2, 128, (5, 24, 32), (5, 6, 8), (2, 3, 4), (1, 2, 2), 0, 3, "block_mean",
+      route_radius=1),
+    # radius two on a 6x6 window grid, float32
+    W("f32_radius2", "f32", 1, 2, 64, (1, 24, 24), (1, 4, 4), (0, 2, 1), (1, 4, 4), 0, 8, "iid", route_radius=2),
 ]
 
 

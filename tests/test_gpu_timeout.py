@@ -19,7 +19,7 @@ def test_bounded_wait_expires_and_context_survives():
 
     wl = synth.Workload("timeout", "bf16", 1, 2, 128, (1, 32, 32), (1, 16, 16), (0, 8, 8), (1, 8, 8), 0, 0, "iid")
     (q, k, v), (qd, kd, vd) = PT.gpu_inputs(wl)
-    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype, route_radius=wl.route_radius)
     out = torch.zeros_like(qd)
     layer.pool_kv(kd, vd, wl.shift)
     layer.attention(qd, kd, vd, out, wl.shift, flags=B.BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD, wait_timeout_us=20000)

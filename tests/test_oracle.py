@@ -99,6 +99,16 @@ def test_pool_constant_field_and_ignores_shift_and_text():
 # ---------------------------------------------------------------- routing
 
 
+def _within_radius(geo, w, u):
+    """Chebyshev distance of window-grid coordinates, computed from scratch."""
+    if geo.route_radius == 0:
+        return True
+    nWt, nWy, nWx = geo.win_grid
+    cw = (w // (nWy * nWx), (w // nWx) % nWy, w % nWx)
+    cu = (u // (nWy * nWx), (u // nWx) % nWy, u % nWx)
+    return max(abs(a - b) for a, b in zip(cw, cu)) <= geo.route_radius
+
+
 def _brute_route(q, k, geo):
     """Explicit loops: window member lists by coordinates, means, scores, sort."""
     T, H, W = geo.grid
@@ -125,7 +135,8 @@ def _brute_route(q, k, geo):
             qm = [q[b, hh, m].mean(axis=0) for m in members]
             km = [k[b, hh, m].mean(axis=0) for m in members]
             for w in range(len(members)):
-                cands = [(-float(np.dot(qm[w], km[u])), u) for u in range(len(members)) if u != w]
+                cands = [(-float(np.dot(qm[w], km[u])), u) for u in range(len(members))
+                         if u != w and _within_radius(geo, w, u)]
                 cands.sort()
                 out[b, hh, w] = [u for _, u in cands[: geo.routed_k]]
     return out
@@ -136,6 +147,9 @@ def _brute_route(q, k, geo):
     [
         O.Geometry(grid=(1, 8, 12), window=(1, 4, 3), shift=(0, 1, 2), routed_k=3),
         O.Geometry(grid=(4, 4, 6), window=(2, 2, 3), shift=(1, 1, 2), routed_k=2),
+        O.Geometry(grid=(1, 12, 15), window=(1, 3, 3), shift=(0, 1, 2), routed_k=3, route_radius=1),
+        O.Geometry(grid=(6, 8, 8), window=(2, 2, 2), shift=(1, 1, 1), routed_k=7, route_radius=1),
+        O.Geometry(grid=(1, 12, 15), window=(1, 2, 3), shift=(0, 1, 2), routed_k=8, route_radius=2),
     ],
 )
 def test_route_matches_brute_force(geo):
@@ -170,6 +184,73 @@ def test_route_ties_go_to_lower_id():
     for w in range(geo.n_win):
         expect = [u for u in range(geo.n_win) if u != w][:4]
         np.testing.assert_array_equal(idx[0, 0, w], expect)
+
+
+def _planted_id_scores(geo):
+    """Q means along e0 everywhere; K mean of window u is u along e0, so the score
+    of u against any query window is proportional to u."""
+    d = 3
+    q = np.zeros((1, 1, geo.N, d))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, geo.N, d))
+    k[0, 0, :, 0] = O.window_of_token(geo).astype(np.float64)
+    return q, k
+
+
+@pytest.mark.parametrize(
+    "geo",
+    [
+        O.Geometry(grid=(1, 16, 16), window=(1, 4, 4), shift=(0, 2, 3), routed_k=1, route_radius=1),
+        O.Geometry(grid=(6, 6, 9), window=(2, 2, 3), shift=(1, 1, 2), routed_k=1, route_radius=1),
+        O.Geometry(grid=(21, 12, 20), window=(21, 3, 4), shift=(0, 1, 2), routed_k=1, route_radius=1),
+    ],
+)
+def test_route_radius_picks_best_neighbour_in_closed_form(geo):
+    """With score(w, u) increasing in u, the best radius-one candidate of window
+    (jt, jy, jx) is the block's far corner (min(j+1, n-1) on every axis), or, for
+    the grid's last window, the window just before it (BASA §A.2: candidate-window
+    radius one). Wrap-around or a one-sided block would pick other windows."""
+    q, k = _planted_id_scores(geo)
+    idx, _ = O.route_windows(q, k, geo)
+    nt, ny, nx = geo.win_grid
+    for w in range(geo.n_win):
+        jt, jy, jx = w // (ny * nx), (w // nx) % ny, w % nx
+        best = (min(jt + 1, nt - 1) * ny + min(jy + 1, ny - 1)) * nx + min(jx + 1, nx - 1)
+        if best == w:  # last window of the grid: the highest other id in its block
+            best = w - 1
+        assert idx[0, 0, w, 0] == best, (w, idx[0, 0, w, 0], best)
+
+
+def test_route_radius_covering_the_grid_equals_global_routing():
+    geo = O.Geometry(grid=(4, 8, 12), window=(2, 2, 3), shift=(1, 1, 2), routed_k=5)
+    q, k, _ = _qkv(geo, B=1, h=2, d=6, seed=5)
+    g0 = O.route_windows(q, k, geo)[0]
+    for r in (max(geo.win_grid) - 1, max(geo.win_grid), 50):
+        g1 = O.route_windows(q, k, O.Geometry(**{**geo.__dict__, "route_radius": r}))[0]
+        np.testing.assert_array_equal(g0, g1)
+
+
+def test_route_radius_candidates_lie_in_the_block():
+    geo = O.Geometry(grid=(1, 20, 24), window=(1, 4, 4), shift=(0, 3, 1), routed_k=3, route_radius=1)
+    q, k, _ = _qkv(geo, B=1, h=3, d=8, seed=9)
+    idx, S = O.route_windows(q, k, geo)
+    for w in range(geo.n_win):
+        n_cand = sum(1 for u in range(geo.n_win) if u != w and _within_radius(geo, w, u))
+        assert np.isfinite(S[0, 0, w]).sum() == n_cand
+        for u in idx[0, :, w].ravel():
+            assert _within_radius(geo, w, int(u)) and u != w
+
+
+def test_full_temporal_windows_ignore_the_temporal_shift():
+    """Windows that span all frames hold the same tokens whatever the temporal shift,
+    and spatial-only pooling ignores the shift: the output cannot depend on st
+    (BASA §3.2 spatial-only pooling and §A.2 full temporal extent, the video setup)."""
+    base = O.Geometry(grid=(4, 6, 8), window=(4, 3, 4), shift=(0, 1, 2), pool=(1, 2, 2), routed_k=1, route_radius=1)
+    q, k, v = _qkv(base, B=1, h=2, d=8, seed=13)
+    ref = O.basa_attention(q, k, v, base)
+    for st in (1, 3):
+        geo = O.Geometry(**{**base.__dict__, "shift": (st, 1, 2)})
+        np.testing.assert_allclose(O.basa_attention(q, k, v, geo), ref, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------- attention
@@ -334,5 +415,10 @@ def test_flop_model_reproduces_table3():
     assert sparse_tf / dense_tf == pytest.approx(rows["basa_w15x26_p4x4"]["tflops"] / rows["dense"]["tflops"], rel=2e-3)
     assert sparse_tf == pytest.approx(rows["basa_w15x26_p4x4"]["tflops"], rel=1e-2)
     assert dense_tf == pytest.approx(rows["dense"]["tflops"], rel=1e-2)
+    # the same count from the video workload's own shape (synth table)
+    from sparse_window_attention_b200 import synth
+    c = A.workload_counts(synth.WORKLOADS["wan_video"])
+    assert c["keys_per_query"] == keys == 24570 and c["N"] == N
+    assert A.sparsity(c["keys_per_query"], c["N"]) == pytest.approx(rows["basa_w15x26_p4x4"]["sparsity"], abs=1e-12)
     for r in rows.values():  # MFU = TFLOPs / latency / 312 TFLOP/s
         assert r["tflops"] / (r["latency_ms"] * 1e-3) / 312.0 == pytest.approx(r["mfu"], abs=6e-5)

@@ -21,7 +21,11 @@ MUTATIONS = [
     ("mask sign", "t = ((np.arange(T) - st) % T) // wt", "t = ((np.arange(T) + st) % T) // wt", ["shift_membership"]),
     ("pool patch stride", "X.reshape(B, h, T // pt, pt, H // ph, ph, W // pw, pw, d)", "X.reshape(B, h, pt, T // pt, ph, H // ph, pw, W // pw, d)", ["pool_centre"]),
     ("route order", "np.lexsort((cand, -sc))", "np.lexsort((cand, sc))", ["route_planted", "route_brute"]),
-    ("route self", ["S[..., np.arange(nw), np.arange(nw)] = -np.inf", "cand = ids[ids != w]"], ["pass", "cand = ids"], ["route_planted", "route_brute"]),
+    ("route self", "return [u for u in range(geo.n_win) if u != w]", "return list(range(geo.n_win))", ["route_planted", "route_brute"]),
+    ("radius wraps", ["for ut in range(max(0, jt - r), min(nt, jt + r + 1)):", "for uy in range(max(0, jy - r), min(ny, jy + r + 1)):", "for ux in range(max(0, jx - r), min(nx, jx + r + 1)):", "u = (ut * ny + uy) * nx + ux"],
+     ["for ut in range(jt - r, jt + r + 1):", "for uy in range(jy - r, jy + r + 1):", "for ux in range(jx - r, jx + r + 1):", "u = ((ut % nt) * ny + uy % ny) * nx + ux % nx"], ["radius_closed_form", "radius_brute"]),
+    ("radius one-sided", "for ux in range(max(0, jx - r), min(nx, jx + r + 1)):", "for ux in range(max(0, jx - r), min(nx, jx + r)):", ["radius_closed_form", "radius_brute"]),
+    ("radius ignores time", "for ut in range(max(0, jt - r), min(nt, jt + r + 1)):", "for ut in range(0, nt):", ["radius_brute"]),
     ("route tie", "np.lexsort((cand, -sc))", "np.lexsort((-cand, -sc))", ["route_ties"]),
     ("drop text keys", "                    kparts.append(k64[b, hh, N:])\n                    vparts.append(v64[b, hh, N:])\n                Kc", "                    pass\n                Kc", ["dense_masked", "constant_scores"]),
     ("drop pooled keys", "                    kparts.append(np.asarray(kp[b, hh], dtype=np.float64))\n                    vparts.append(np.asarray(vp[b, hh], dtype=np.float64))\n                if geo.n_text > 0:\n                    kparts.append(k64[b, hh, N:])", "                    pass\n                if geo.n_text > 0:\n                    kparts.append(k64[b, hh, N:])", ["dense_masked"]),
@@ -37,6 +41,12 @@ PINS = {
     "route_planted": lambda: pins.test_route_planted_winner_and_self_excluded(),
     "route_brute": lambda: [pins.test_route_matches_brute_force(g) for g in (pins.O.Geometry(grid=(1, 8, 12), window=(1, 4, 3), shift=(0, 1, 2), routed_k=3),)],
     "route_ties": lambda: pins.test_route_ties_go_to_lower_id(),
+    "radius_closed_form": lambda: [pins.test_route_radius_picks_best_neighbour_in_closed_form(g) for g in (
+        pins.O.Geometry(grid=(1, 16, 16), window=(1, 4, 4), shift=(0, 2, 3), routed_k=1, route_radius=1),
+        pins.O.Geometry(grid=(6, 6, 9), window=(2, 2, 3), shift=(1, 1, 2), routed_k=1, route_radius=1))],
+    "radius_brute": lambda: [pins.test_route_matches_brute_force(g) for g in (
+        pins.O.Geometry(grid=(1, 12, 15), window=(1, 3, 3), shift=(0, 1, 2), routed_k=3, route_radius=1),
+        pins.O.Geometry(grid=(6, 8, 8), window=(2, 2, 2), shift=(1, 1, 1), routed_k=7, route_radius=1))],
     "dense_masked": lambda: [pins.test_attention_matches_dense_masked_brute_force(g) for g in pins.TINY_GEOS],
     "constant_scores": lambda: [pins.test_constant_scores_give_mean_of_key_values(g) for g in pins.TINY_GEOS],
     "closed_form": lambda: pins.test_closed_form_whole_grid_is_dense_sdpa(),
