@@ -159,15 +159,19 @@ def run_ours(args, world, rank, local):
     out = torch.empty_like(qd)
     stream = torch.cuda.current_stream()
 
+    fused = layer.fused and all(layer.fused_bytes(sh) > 0 for sh in shifts)
+
     def step(i, ev=None):
         sh = shifts[i % len(shifts)]
         if ev is not None:
             ev[0].record(stream)
-        if layer.has_pool:
+        if fused:  # pooled K/V and routing in one pass over q, k, v
+            layer.pool_route(qd, kd, vd, sh)
+        elif layer.has_pool:
             layer.pool_kv(kd, vd, sh)
         if ev is not None:
             ev[1].record(stream)
-        if layer.routed_k > 0:
+        if layer.routed_k > 0 and not fused:
             layer.route(qd, kd, sh)
         if ev is not None:
             ev[2].record(stream)
@@ -251,14 +255,7 @@ def run_ours(args, world, rank, local):
             "traffic": traffic,
             "attn_ms": round(attn_ms, 4),
         },
-        "hbm_kernels": {
-            "pool_kv": {"ms": round(pool_ms, 4), "bytes": cnt["pool_bytes"],
-                        "GB/s": round(cnt["pool_bytes"] / (pool_ms * 1e-3) / 1e9, 1) if cnt["pool_bytes"] else None,
-                        "frac_of_measured_hbm": round(cnt["pool_bytes"] / (pool_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if cnt["pool_bytes"] else None},
-            "route": {"ms": round(route_ms, 4), "bytes": cnt["route_bytes"],
-                      "GB/s": round(cnt["route_bytes"] / (route_ms * 1e-3) / 1e9, 1) if cnt["route_bytes"] else None,
-                      "frac_of_measured_hbm": round(cnt["route_bytes"] / (route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if cnt["route_bytes"] else None},
-        },
+        "hbm_kernels": hbm_lines(cnt, pool_ms, route_ms, peaks["hbm_gbs"], fused),
         "clocks": clocks,
         "gpu_launches": args.steps * layer.launches_per_forward(),
     }
@@ -269,6 +266,23 @@ def run_ours(args, world, rank, local):
             if args.workload != name:
                 res["also_" + name] = run_also(args, name)
     return res
+
+
+def hbm_lines(cnt, pool_ms, route_ms, hbm_gbs, fused):
+    """Achieved bandwidth of the HBM-bound pre-pass: compulsory bytes / event time."""
+    def line(ms, nbytes, what):
+        if not nbytes:
+            return None
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": round(ms, 4), "bytes": nbytes, "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm_gbs, 4),
+                "launches": what}
+
+    if fused:
+        # one read of q, k, v + pooled K/V written; partial sums and top-k are inside the time
+        return {"pool_route_fused": line(pool_ms, cnt["pool_route_bytes"],
+                                         "pool + window partial sums, partial reduction, top-k")}
+    return {"pool_kv": line(pool_ms, cnt["pool_bytes"], "box means over pool patches"),
+            "route": line(route_ms, cnt["route_bytes"], "box means over windows, top-k")}
 
 
 def run_e2e(args, layer, q, k, v, shifts, flops, world):

@@ -139,6 +139,28 @@ basa_status basa_route_windows(const void *q, const void *k, int32_t *route_idx,
                                const basa_params *p, basa_stream_t stream);
 
 /*
+ * basa_pool_route — basa_pool_kv followed by basa_route_windows, fused into one
+ * read of q, k and v (BASA §3.2 pooled global K/V, §3.3 routing; the pages run
+ * them as separate reductions, this pass shares the reads).
+ *
+ * Same results as the two calls: kp, vp as basa_pool_kv (float32 sums, one
+ * rounding), route_idx / route_score as basa_route_windows (the window means are
+ * summed in another fixed order, so float32 scores can differ in the last bits).
+ * Requires a pool patch and routed_k >= 1. `workspace` is a device buffer of at
+ * least basa_pool_route_workspace_bytes(p) bytes, 16-byte aligned; its contents
+ * on entry are ignored; on return it starts with the window means
+ * [2][B][heads][nWin][head_dim] (float32), followed by per-box partial sums.
+ * Returns BASA_ERR_UNSUPPORTED when the shape does not fit the fused kernel
+ * (then basa_pool_route_workspace_bytes returns 0); the two separate calls
+ * accept every shape this one rejects for that reason.
+ */
+size_t basa_pool_route_workspace_bytes(const basa_params *p);
+basa_status basa_pool_route(const void *q, const void *k, const void *v,
+                            void *kp, void *vp, int32_t *route_idx,
+                            float *route_score, void *workspace,
+                            const basa_params *p, basa_stream_t stream);
+
+/*
  * basa_window_attn_fwd — shifted-window attention forward (BASA §3.1 shifted
  * windows; §A.1: the local and global/text branches equal ONE softmax over the
  * concatenated K/V, which is what is computed here in a single pass).

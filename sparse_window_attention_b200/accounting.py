@@ -52,6 +52,8 @@ def workload_counts(wl) -> dict:
         "pool_bytes": bh * (2 * N * row + 2 * n_pool * row) if n_pool else 0,
         # route: read visual Q and K (the window means and scores are negligible)
         "route_bytes": bh * 2 * N * row if wl.routed_k > 0 else 0,
+        # fused pool + routing pass: read visual Q, K, V once, write Kp and Vp
+        "pool_route_bytes": bh * (3 * N * row + 2 * n_pool * row) if (n_pool and wl.routed_k > 0) else 0,
         # attention: read Q, K, V (visual + text), Kp, Vp; write O
         "attn_bytes": bh * row * (N + 2 * (N + wl.n_text) + 2 * n_pool + N),
     }

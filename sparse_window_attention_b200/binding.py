@@ -30,6 +30,8 @@ EXPORTED = (
     "basa_route_workspace_bytes",
     "basa_route_windows",
     "basa_route_windows_noalloc",
+    "basa_pool_route_workspace_bytes",
+    "basa_pool_route",
     "basa_window_attn_fwd",
     "basa_status_string",
     "basa_device_error_status",
@@ -72,6 +74,10 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.basa_route_windows.restype = ctypes.c_int
     lib.basa_route_windows_noalloc.argtypes = [vp, vp, vp, vp, P, vp]
     lib.basa_route_windows_noalloc.restype = ctypes.c_int
+    lib.basa_pool_route_workspace_bytes.argtypes = [P]
+    lib.basa_pool_route_workspace_bytes.restype = ctypes.c_size_t
+    lib.basa_pool_route.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, P, vp]
+    lib.basa_pool_route.restype = ctypes.c_int
     lib.basa_window_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, P, vp]
     lib.basa_window_attn_fwd.restype = ctypes.c_int
     lib.basa_status_string.argtypes = [ctypes.c_int]
@@ -156,6 +162,19 @@ def basa_route_windows_noalloc(q, k, route_idx, route_score, params: basa_params
                                          ctypes.byref(params), _stream(stream))
     if check:
         _check(st, "basa_route_windows_noalloc")
+    return st
+
+
+def basa_pool_route_workspace_bytes(params: basa_params) -> int:
+    return _lib.basa_pool_route_workspace_bytes(ctypes.byref(params))
+
+
+def basa_pool_route(q, k, v, kp, vp, route_idx, route_score, workspace, params: basa_params, stream=None,
+                    check=True) -> int:
+    st = _lib.basa_pool_route(_ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp), _ptr(route_idx), _ptr(route_score),
+                              _ptr(workspace), ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_pool_route")
     return st
 
 

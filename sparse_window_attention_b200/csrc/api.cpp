@@ -119,6 +119,33 @@ basa_status basa_route_windows_noalloc(const void *q, const void *k, int32_t *ro
   return basa::launch_route_noalloc(q, k, route_idx, route_score, *p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t basa_pool_route_workspace_bytes(const basa_params *p) {
+  if (check_common(p) != BASA_OK || !has_pool(p) || p->routed_k < 1) return 0;
+  basa::FusedPlan fp;
+  if (basa::plan_fused(*p, &fp) != BASA_OK) return 0;
+  return fp.means_bytes + fp.part_bytes;
+}
+
+basa_status basa_pool_route(const void *q, const void *k, const void *v, void *kp, void *vp, int32_t *route_idx,
+                            float *route_score, void *workspace, const basa_params *p, basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (!has_pool(p) || p->routed_k < 1) return BASA_ERR_INVALID_ARG;
+  const int64_t nwin = int64_t(p->T / p->wt) * (p->H / p->wh) * (p->W / p->ww);
+  if (nwin > 4096) return BASA_ERR_UNSUPPORTED;
+  basa::FusedPlan fp;
+  st = basa::plan_fused(*p, &fp);
+  if (st != BASA_OK) return st;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q || !k || !v || !kp || !vp || !route_idx || !workspace) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kp) || !aligned16(vp) || !aligned16(workspace) ||
+      !aligned4(route_idx))
+    return BASA_ERR_INVALID_ARG;
+  if (route_score && !aligned4(route_score)) return BASA_ERR_INVALID_ARG;
+  return basa::launch_pool_route_fused(q, k, v, kp, vp, route_idx, route_score, workspace, *p,
+                                       reinterpret_cast<cudaStream_t>(stream));
+}
+
 basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                                  const int32_t *route_idx, void *out, const basa_params *p,
                                  basa_stream_t stream) {

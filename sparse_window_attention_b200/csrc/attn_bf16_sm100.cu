@@ -605,18 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encoder(); }
 
 // 5-D map (d, x, y, t, b*head) over the visual rows of a [B, heads, rows, 128] tensor.
 bool encode_grid_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh,
@@ -646,6 +635,19 @@ bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, lon
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
 
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                              const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s) {

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -92,6 +93,30 @@ __host__ __device__ inline void window_origin(const Geo &g, int w, int *ot, int 
   *type = (*ot + g.wt > g.T ? 1 : 0) | (*oy + g.wh > g.H ? 2 : 0) | (*ox + g.ww > g.W ? 4 : 0);
 }
 
+// Driver entry point that encodes TMA tensor maps (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// ---------------------------------------------------------------------------
+// Fused pooling + window-mean pass (one read of Q, K and V).
+//
+// The grid is cut into boxes of e = m * pool-patch tokens per axis (whole pool
+// patches, so pooled K/V are complete inside one box). Every box writes its
+// pooled K/V and, for each window it meets, the partial sums of Q and K over
+// box ∩ window into a slot of its own; a second kernel adds each window's slots
+// in a fixed order. Window u meets boxes b0(u), b0(u)+1, ... (mod boxes per axis)
+// along each axis, b0 = floor(origin / e), and its slot along that axis is the
+// box's position in that run.
+struct FusedPlan {
+  int e[3];       // box extents (t, y, x)
+  int nb[3];      // boxes per axis
+  int K[3];       // slots per window per axis
+  int max_cells;  // upper bound on the cells (patch ∩ window pieces) of a box
+  size_t means_bytes;  // window means of Q and K: 2 * B*heads * nWin * head_dim floats
+  size_t part_bytes;   // partial slots: 2 * B*heads * nWin * K[0]*K[1]*K[2] * head_dim floats
+};
+// BASA_OK, or BASA_ERR_UNSUPPORTED when no box fits the kernel's limits.
+basa_status plan_fused(const basa_params &p, FusedPlan *fp);
+
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns BASA_OK or BASA_ERR_CUDA).
 // ---------------------------------------------------------------------------
@@ -101,6 +126,12 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
 // Routing with the library's fixed device scratch array instead of a workspace.
 basa_status launch_route_noalloc(const void *q, const void *k, int32_t *route_idx, float *route_score,
                                  const basa_params &p, cudaStream_t s);
+// Top-k over window means qm, km ([B*heads][nWin][head_dim] float each).
+basa_status launch_topk(const float *qm, const float *km, int32_t *route_idx, float *route_score, const basa_params &p,
+                        cudaStream_t s);
+// Fused pooling + window means + top-k; `workspace` holds means_bytes + part_bytes.
+basa_status launch_pool_route_fused(const void *q, const void *k, const void *v, void *kp, void *vp, int32_t *route_idx,
+                                    float *route_score, void *workspace, const basa_params &p, cudaStream_t s);
 basa_status launch_attn_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                             const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,

@@ -315,6 +315,13 @@ basa_status launch_route(const void *q, const void *k, int32_t *route_idx, float
   a.inv_count = 1.0f / float(p.wt * p.wh * p.ww);
   basa_status st = (p.dtype == BASA_BF16) ? run_box_mean<__nv_bfloat16, float>(a, bh, s) : run_box_mean<float, float>(a, bh, s);
   if (st != BASA_OK) return st;
+  return launch_topk(qm, km, route_idx, route_score, p, s);
+}
+
+basa_status launch_topk(const float *qm, const float *km, int32_t *route_idx, float *route_score, const basa_params &p,
+                        cudaStream_t s) {
+  const Geo g = make_geo(p);
+  const int bh = p.B * p.heads;
   RouteArgs r{qm, km, route_idx, route_score, g.nWin, p.head_dim, p.routed_k, p.route_radius, g.nWy, g.nWx};
   const size_t smem = (size_t(kRouteChunk) * (p.head_dim + 4) + kRouteWarps * p.head_dim + size_t(kRouteWarps) * g.nWin) * sizeof(float);
   static bool attr_set[64] = {false};

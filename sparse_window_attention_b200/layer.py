@@ -38,6 +38,10 @@ class BasaLayer:
             self.route_score = torch.empty(batch, heads, self.n_win, routed_k, dtype=torch.float32, device=self.device)
             nbytes = B.basa_route_workspace_bytes(self.params((0, 0, 0)))
             self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+        # fused pooling + routing pass (one read of q, k, v) where the shape allows it;
+        # its workspace size depends on the shift and grows on first use
+        self.fused = self.has_pool and routed_k > 0
+        self.fused_workspace = None
 
     def params(self, shift, **extra) -> B.basa_params:
         key = (tuple(shift), tuple(sorted(extra.items())))
@@ -53,6 +57,17 @@ class BasaLayer:
     def route(self, q, k, shift, stream=None):
         B.basa_route_windows(q, k, self.route_idx, self.route_score, self.workspace, self.params(shift), stream)
 
+    def fused_bytes(self, shift) -> int:
+        return B.basa_pool_route_workspace_bytes(self.params(shift))
+
+    def pool_route(self, q, k, v, shift, stream=None):
+        """Pooled K/V and routed windows in one pass (basa_pool_route)."""
+        nbytes = self.fused_bytes(shift)
+        if self.fused_workspace is None or self.fused_workspace.numel() < nbytes:
+            self.fused_workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+        B.basa_pool_route(q, k, v, self.kp, self.vp, self.route_idx, self.route_score, self.fused_workspace,
+                          self.params(shift), stream)
+
     def attention(self, q, k, v, out, shift, kp=None, vp=None, route_idx=None, stream=None, **extra):
         kp = self.kp if kp is None else kp
         vp = self.vp if vp is None else vp
@@ -63,14 +78,18 @@ class BasaLayer:
         """Full layer: pooled K/V, routed windows (if routed_k > 0), attention."""
         if out is None:
             out = torch.empty_like(q)
-        if self.has_pool:
-            self.pool_kv(k, v, shift, stream)
-        if self.routed_k > 0:
-            self.route(q, k, shift, stream)
+        if self.fused and self.fused_bytes(shift) > 0:
+            self.pool_route(q, k, v, shift, stream)
+        else:
+            if self.has_pool:
+                self.pool_kv(k, v, shift, stream)
+            if self.routed_k > 0:
+                self.route(q, k, shift, stream)
         self.attention(q, k, v, out, shift, stream=stream)
         return out
 
     def launches_per_forward(self) -> int:
+        # fused: pool + partial sums, reduction, top-k; else pool, means + top-k
         return (1 if self.has_pool else 0) + (2 if self.routed_k > 0 else 0) + 1
 
     def device_error(self) -> int:

@@ -119,6 +119,28 @@ def test_route_radius_limits_routed_k():
     assert B.basa_route_workspace_bytes(p) == 2 * 12 * 16 * 128 * 4
 
 
+def test_fused_pool_route_checks():
+    """basa_pool_route: needs pooling and routing; shapes whose boxes would hold too
+    many pieces (pool patch ∩ window) are refused before any launch."""
+    pr = _p(routed_k=2)
+    n = B.basa_pool_route_workspace_bytes(pr)
+    # window means (2 x heads x 16 windows x 128 floats) + at least one partial slot each
+    assert n >= 2 * (2 * 2 * 16 * 128 * 4)
+    assert B.basa_pool_route_workspace_bytes(_p()) == 0  # no routing
+    assert B.basa_pool_route_workspace_bytes(_p(routed_k=2, pool=(0, 0, 0))) == 0
+    assert B.basa_pool_route(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, _p(), stream=0, check=False) == 1
+    # a 32x32 patch cut by 2x2 windows into 256 cells: more than one CTA may hold
+    big = _p(routed_k=2, pool=(1, 32, 32), window=(1, 2, 2), shift=(0, 1, 1))
+    assert B.basa_pool_route_workspace_bytes(big) == 0
+    assert B.basa_pool_route(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, big, stream=0, check=False) == 3
+    # null and misaligned pointers
+    assert B.basa_pool_route(FAKE, FAKE, None, FAKE, FAKE, FAKE, None, FAKE, pr, stream=0, check=False) == 1
+    assert B.basa_pool_route(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE + 4, pr, stream=0, check=False) == 1
+    # the video configuration fits
+    p = B.make_params(1, 12, 128, (21, 60, 104), (21, 15, 26), (0, 7, 13), (1, 4, 4), 0, 1, "bf16", route_radius=1)
+    assert B.basa_pool_route_workspace_bytes(p) > 2 * 12 * 16 * 128 * 4
+
+
 def test_route_workspace_bytes():
     p = _p(routed_k=2)
     assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4

@@ -179,6 +179,76 @@ def test_wan_video_full_size(shift):
     frames, spatial-only 4x4 pooling, one routed window among radius-one neighbours."""
     differing = run_sampled_parity(synth.WORKLOADS["wan_video"], shift)
     assert differing == 0
+
+
+# ----------------------------------------------------------------- fused pool + routing pass
+
+
+def run_fused_parity(wl, shift, seed=0, large=False):
+    """basa_pool_route (one read of q, k, v) against the oracle's pooling and routing."""
+    from sparse_window_attention_b200 import binding as B
+
+    if large:
+        (qd, kd, vd), (q64, k64, v64) = _large_inputs(wl, seed)
+    else:
+        (q, k, v), (qd, kd, vd) = PT.gpu_inputs(wl, seed)
+        hs0 = _heads(wl)
+        q64, k64, v64 = PT.to64(q[:, hs0]), PT.to64(k[:, hs0]), PT.to64(v[:, hs0])
+    geo = PT.geometry(wl, shift)
+    hs = _heads(wl)
+    layer = _layer(wl)
+    assert layer.fused_bytes(shift) > 0, "shape not supported by the fused pass"
+    layer.kp.fill_(float("nan"))
+    layer.vp.fill_(float("nan"))
+    layer.route_idx.fill_(-1)
+    layer.pool_route(qd, kd, vd, shift)
+    torch.cuda.synchronize()
+    assert not torch.isnan(layer.kp).any() and not torch.isnan(layer.vp).any()
+    kp_ex, vp_ex = O.pool_kv(k64, v64, geo)
+    PT.assert_pool_close(PT.to64(layer.kp[:, hs]), kp_ex, wl.dtype)
+    PT.assert_pool_close(PT.to64(layer.vp[:, hs]), vp_ex, wl.dtype)
+    route_or, S = O.route_windows(q64, k64, geo)
+    differing = PT.check_routes(layer.route_idx[:, hs].cpu().numpy(), route_or, S)
+    gs = layer.route_score[:, hs].cpu().numpy().astype(np.float64)
+    ref = np.take_along_axis(S, layer.route_idx[:, hs].cpu().numpy().astype(np.int64), axis=3)
+    assert np.all(np.abs(gs - ref) <= PT.ROUTE_SCORE_TOL * np.maximum(1.0, np.abs(ref)))
+    # the window means at the head of the workspace match the oracle's
+    T, H, W = wl.grid
+    nwin = geo.n_win
+    means = layer.fused_workspace[: 2 * wl.B * wl.heads * nwin * wl.d * 4].view(torch.float32)
+    means = means.view(2, wl.B, wl.heads, nwin, wl.d)[:, :, hs].cpu().numpy().astype(np.float64)
+    qm, km = O.window_means(q64, k64, geo)
+    np.testing.assert_allclose(means[0], qm, rtol=0, atol=1e-5 * max(1.0, np.abs(qm).max()))
+    np.testing.assert_allclose(means[1], km, rtol=0, atol=1e-5 * max(1.0, np.abs(km).max()))
+    return differing
+
+
+FUSED = [
+    W("wrap3d", "bf16", 1, 2, 128, (4, 8, 12), (2, 4, 4), (1, 2, 3), (2, 4, 4), 0, 11, "block_mean"),
+    W("odd", "bf16", 2, 2, 128, (3, 12, 26), (3, 6, 13), (0, 3, 6), (3, 6, 13), 5, 2, "block_mean"),
+    W("rows", "bf16", 1, 2, 128, (1, 4, 80), (1, 1, 40), (0, 1, 17), (1, 2, 8), 0, 1, "iid"),
+    # window wider than the box on every axis, the box spanning the whole t axis
+    W("whole_t", "bf16", 1, 2, 128, (5, 24, 32), (5, 6, 8), (2, 3, 4), (5, 2, 2), 0, 3, "block_mean", route_radius=1),
+    # pool patches larger than windows along x, pooled box wider than the grid's windows
+    W("wide_pool", "bf16", 1, 2, 128, (2, 16, 48), (1, 4, 6), (1, 1, 5), (2, 4, 12), 3, 2, "iid"),
+    W("f32_d128", "f32", 1, 2, 128, (2, 16, 16), (1, 8, 8), (1, 4, 2), (2, 4, 4), 9, 2, "block_mean"),
+    W("f32_d64", "f32", 2, 3, 64, (1, 24, 16), (1, 8, 8), (0, 5, 3), (1, 4, 4), 0, 1, "iid"),
+    W("bf16_d64", "bf16", 1, 2, 64, (1, 24, 16), (1, 8, 8), (0, 5, 3), (1, 4, 4), 0, 1, "iid"),
+]
+
+
+@pytest.mark.parametrize("wl", FUSED, ids=[w.name for w in FUSED])
+def test_fused_pool_route_small(wl):
+    run_fused_parity(wl, wl.shift)
+
+
+def test_fused_pool_route_wan():
+    assert run_fused_parity(synth.WORKLOADS["wan"], (0, 3, 6)) == 0
+
+
+@pytest.mark.parametrize("shift", synth.SHIFT_CYCLES["wan_video"])
+def test_fused_pool_route_wan_video(shift):
+    assert run_fused_parity(synth.WORKLOADS["wan_video"], shift, large=True) == 0
     if shift == synth.SHIFT_CYCLES["wan_video"][-1]:
         _LARGE.clear()
 
