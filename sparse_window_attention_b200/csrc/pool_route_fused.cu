@@ -334,46 +334,55 @@ struct ReduceArgs {
   const float *part;
   float *means;  // [2][bh][nWin][d]
   int d, bh;
+  int groups;    // threads adding one window's slots per column
   int G[3], e[3], nb[3], w[3], s[3], nw[3], K[3];
   float inv_win;
 };
 
-// One CTA per (tensor, b*head, window): thread (float4 column c4, group g) adds
-// the window's slots g, g + G, ... (G = 256 / (d/4)); the G group sums are then
-// added in group order.
+// CTA of 256 threads = `wpc` windows x `groups` x (d/4) float4 columns: thread
+// (window, group g, column c4) adds the window's slots g, g + groups, ...; the
+// group sums are then added in group order. Windows with few slots take one
+// group (several windows per CTA), windows with many slots take up to eight.
 __global__ void __launch_bounds__(256) window_reduce_kernel(const __grid_constant__ ReduceArgs a) {
   __shared__ float4 red[256];
   const int d4 = a.d / 4;
-  const int groups = blockDim.x / d4;
+  const int groups = a.groups;
+  const int wpc = blockDim.x / (d4 * groups);
   const int nWin = a.nw[0] * a.nw[1] * a.nw[2];
-  const int row = blockIdx.x;  // (tensor, bh, window)
-  const int win = row % nWin;
-  const int c4 = threadIdx.x % d4, g = threadIdx.x / d4;
-  const int j[3] = {win / (a.nw[1] * a.nw[2]), (win / a.nw[2]) % a.nw[1], win % a.nw[2]};
-  int n[3];
-#pragma unroll
-  for (int ax = 0; ax < 3; ++ax) {
-    const int o = (j[ax] * a.w[ax] + a.s[ax]) % a.G[ax];
-    n[ax] = min((o + a.w[ax] - 1) / a.e[ax] - o / a.e[ax] + 1, a.nb[ax]);
-  }
-  const float4 *p = reinterpret_cast<const float4 *>(a.part) + (long long)row * a.K[0] * a.K[1] * a.K[2] * d4 + c4;
+  const int local = threadIdx.x / (d4 * groups);
+  const int g = (threadIdx.x / d4) % groups, c4 = threadIdx.x % d4;
+  const int row = blockIdx.x * wpc + local;  // (tensor, bh, window)
+  const bool valid = row < 2 * a.bh * nWin;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int total = n[0] * n[1] * n[2];
-  for (int i = g; i < total; i += groups) {
-    const int kx = i % n[2], ky = (i / n[2]) % n[1], kt = i / (n[2] * n[1]);
-    const float4 v = p[(((long long)kt * a.K[1] + ky) * a.K[2] + kx) * d4];
-    s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-  }
-  red[threadIdx.x] = s;
-  __syncthreads();
-  if (g == 0) {
-    for (int h = 1; h < groups; ++h) {
-      const float4 v = red[h * d4 + c4];
+  if (valid) {
+    const int win = row % nWin;
+    const int j[3] = {win / (a.nw[1] * a.nw[2]), (win / a.nw[2]) % a.nw[1], win % a.nw[2]};
+    int n[3];
+#pragma unroll
+    for (int ax = 0; ax < 3; ++ax) {
+      const int o = (j[ax] * a.w[ax] + a.s[ax]) % a.G[ax];
+      n[ax] = min((o + a.w[ax] - 1) / a.e[ax] - o / a.e[ax] + 1, a.nb[ax]);
+    }
+    const float4 *p = reinterpret_cast<const float4 *>(a.part) + (long long)row * a.K[0] * a.K[1] * a.K[2] * d4 + c4;
+    const int total = n[0] * n[1] * n[2];
+    for (int i = g; i < total; i += groups) {
+      const int kx = i % n[2], ky = (i / n[2]) % n[1], kt = i / (n[2] * n[1]);
+      const float4 v = p[(((long long)kt * a.K[1] + ky) * a.K[2] + kx) * d4];
       s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
     }
+  }
+  if (groups > 1) {
+    red[threadIdx.x] = s;
+    __syncthreads();
+    if (g == 0)
+      for (int h = 1; h < groups; ++h) {
+        const float4 v = red[threadIdx.x + h * d4];
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+  }
+  if (valid && g == 0)
     reinterpret_cast<float4 *>(a.means)[(long long)row * d4 + c4] =
         make_float4(s.x * a.inv_win, s.y * a.inv_win, s.z * a.inv_win, s.w * a.inv_win);
-  }
 }
 
 }  // namespace
@@ -501,8 +510,14 @@ basa_status launch_pool_route_fused(const void *q, const void *k, const void *v,
     r.s[ax] = a.s[ax]; r.nw[ax] = a.nw[ax]; r.K[ax] = a.K[ax];
   }
   r.inv_win = 1.0f / float(p.wt * p.wh * p.ww);
-  const int reduce_threads_per_cta = (256 / (p.head_dim / 4)) * (p.head_dim / 4);
-  window_reduce_kernel<<<unsigned(2ll * a.bh * g.nWin), reduce_threads_per_cta, 0, s>>>(r);
+  // about 8 slots per thread; groups divide 256 / (d/4)
+  const int d4 = p.head_dim / 4;
+  const int kprod = fp.K[0] * fp.K[1] * fp.K[2];
+  r.groups = 1;
+  while (r.groups * 2 <= 256 / d4 && r.groups * 8 < kprod) r.groups *= 2;
+  const int wpc = 256 / (d4 * r.groups);
+  const long long rows = 2ll * a.bh * g.nWin;
+  window_reduce_kernel<<<unsigned((rows + wpc - 1) / wpc), 256, 0, s>>>(r);
   if (cudaGetLastError() != cudaSuccess) return BASA_ERR_CUDA;
   const size_t half = fp.means_bytes / 2;
   return launch_topk(means, reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(means) + half), route_idx, route_score,
