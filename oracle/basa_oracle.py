@@ -23,6 +23,9 @@ blocking, fusion or reordering beyond what the definition needs:
    branches are equivalent to one softmax over concatenated K/V);
 6. inverse shift of the output.
 
+The branch form (branch_attention, merge_branches) evaluates key groups separately
+with their log-sum-exp and merges them (BASA §A.1).
+
 Readings taken where the pages are silent:
   * shift convention Xr[t,y,x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W] (roll by -s);
   * window ids are raster order over the window grid of the shifted frame;
@@ -268,6 +271,76 @@ def basa_attention(q, k, v, geo: Geometry, kp=None, vp=None, route_idx=None, ret
                 Ow[b, hh, w] = p @ Vc
     O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)
     return O.reshape(B, h, N, d)
+
+
+# Key groups of the branch form (BASA §A.1: the local-window and text/global-memory
+# branches can be evaluated separately; the result equals one softmax over all keys).
+KEYS_WINDOWS = 1  # own window and routed windows
+KEYS_POOLED = 2
+KEYS_TEXT = 4
+KEYS_ALL = KEYS_WINDOWS | KEYS_POOLED | KEYS_TEXT
+
+
+def branch_attention(q, k, v, geo: Geometry, keys, kp=None, vp=None, route_idx=None):
+    """One branch of the decomposed form: attention of every query over the key
+    groups in ``keys`` only, and the log-sum-exp of its scaled scores.
+
+    out_i = sum_j softmax_j(s_ij) v_j and lse_i = log sum_j exp(s_ij), with
+    s_ij = q_i . k_j / sqrt(d) over the selected groups (BASA §A.1). Returns
+    (out [B, h, N, d], lse [B, h, N]) float64, both at original token positions.
+    """
+    q64 = np.asarray(q, dtype=np.float64)
+    k64 = np.asarray(k, dtype=np.float64)
+    v64 = np.asarray(v, dtype=np.float64)
+    B, h, N, d = q64.shape
+    if geo.has_pool and kp is None:
+        kp, vp = pool_kv(k64, v64, geo)
+    if geo.routed_k > 0 and route_idx is None:
+        route_idx, _ = route_windows(q64, k64, geo)
+
+    def windows(x):
+        return window_partition(cyclic_shift(to_grid(x[:, :, :N], geo.grid), geo.shift), geo.window)
+
+    Qw, Kw, Vw = windows(q64), windows(k64), windows(v64)
+    Ow = np.empty_like(Qw)
+    Lw = np.empty(Qw.shape[:-1])
+    scale = 1.0 / np.sqrt(d)
+    for b in range(B):
+        for hh in range(h):
+            for w in range(geo.n_win):
+                kparts, vparts = [], []
+                if keys & KEYS_WINDOWS:
+                    for u in [w] + [int(route_idx[b, hh, w, r]) for r in range(geo.routed_k)]:
+                        kparts.append(Kw[b, hh, u])
+                        vparts.append(Vw[b, hh, u])
+                if keys & KEYS_POOLED and geo.has_pool:
+                    kparts.append(np.asarray(kp[b, hh], dtype=np.float64))
+                    vparts.append(np.asarray(vp[b, hh], dtype=np.float64))
+                if keys & KEYS_TEXT and geo.n_text > 0:
+                    kparts.append(k64[b, hh, N:])
+                    vparts.append(v64[b, hh, N:])
+                Kc = np.concatenate(kparts, axis=0)
+                Vc = np.concatenate(vparts, axis=0)
+                s = (Qw[b, hh, w] @ Kc.T) * scale
+                m = s.max(axis=1, keepdims=True)
+                e = np.exp(s - m)
+                l = e.sum(axis=1, keepdims=True)
+                Ow[b, hh, w] = (e / l) @ Vc
+                Lw[b, hh, w] = (m + np.log(l))[:, 0]
+    O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)
+    L = inverse_cyclic_shift(window_unpartition(Lw[..., None], geo.grid, geo.window), geo.shift)
+    return O.reshape(B, h, N, d), L.reshape(B, h, N)
+
+
+def merge_branches(outs, lses):
+    """Merge branch results into the joint softmax (BASA §A.1): with L = log sum_b
+    exp(lse_b), out = sum_b exp(lse_b - L) out_b. Returns (out, L)."""
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])
+    m = L.max(axis=0)
+    wts = np.exp(L - m)
+    tot = wts.sum(axis=0)
+    out = sum(wts[i][..., None] * np.asarray(outs[i], dtype=np.float64) for i in range(len(outs))) / tot[..., None]
+    return out, m + np.log(tot)
 
 
 def window_of_token(geo: Geometry):

@@ -422,3 +422,54 @@ def test_flop_model_reproduces_table3():
     assert A.sparsity(c["keys_per_query"], c["N"]) == pytest.approx(rows["basa_w15x26_p4x4"]["sparsity"], abs=1e-12)
     for r in rows.values():  # MFU = TFLOPs / latency / 312 TFLOP/s
         assert r["tflops"] / (r["latency_ms"] * 1e-3) / 312.0 == pytest.approx(r["mfu"], abs=6e-5)
+
+
+# ---------------------------------------------------------------- branch form (LSE)
+
+
+@pytest.mark.parametrize("geo", TINY_GEOS)
+def test_branches_merge_to_the_joint_softmax(geo):
+    """BASA §A.1: local and text/global branches evaluated separately equal one
+    softmax over the concatenated keys; two-way and three-way splits."""
+    q, k, v = _qkv(geo, B=1, h=2, d=8, seed=21)
+    route = O.route_windows(q, k, geo)[0] if geo.routed_k else None
+    joint = O.basa_attention(q, k, v, geo, route_idx=route)
+    out_all, lse_all = O.branch_attention(q, k, v, geo, O.KEYS_ALL, route_idx=route)
+    np.testing.assert_allclose(out_all, joint, rtol=0, atol=1e-12)
+    glob = (O.KEYS_POOLED if geo.has_pool else 0) | (O.KEYS_TEXT if geo.n_text else 0)
+    if not glob:
+        return
+    splits = [[O.KEYS_WINDOWS, glob]]
+    if geo.has_pool and geo.n_text:
+        splits.append([O.KEYS_WINDOWS, O.KEYS_POOLED, O.KEYS_TEXT])
+    for parts in splits:
+        res = [O.branch_attention(q, k, v, geo, keys, route_idx=route) for keys in parts]
+        out, lse = O.merge_branches([r[0] for r in res], [r[1] for r in res])
+        np.testing.assert_allclose(out, joint, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_all, rtol=0, atol=1e-12)
+
+
+def test_lse_of_zero_queries_is_log_of_key_count():
+    """q = 0: every score is 0, so lse = log(number of keys) exactly."""
+    geo = TINY_GEOS[0]
+    q, k, v = _qkv(geo, B=1, h=1, d=8, seed=2)
+    q[:] = 0.0
+    route = O.route_windows(q, k, geo)[0]
+    n_keys = geo.win_tokens * (1 + geo.routed_k) + geo.n_pool + geo.n_text
+    _, lse = O.branch_attention(q, k, v, geo, O.KEYS_ALL, route_idx=route)
+    np.testing.assert_allclose(lse, np.log(n_keys), rtol=0, atol=1e-12)
+    _, lse_w = O.branch_attention(q, k, v, geo, O.KEYS_WINDOWS, route_idx=route)
+    np.testing.assert_allclose(lse_w, np.log(geo.win_tokens * (1 + geo.routed_k)), rtol=0, atol=1e-12)
+
+
+def test_lse_whole_grid_is_scipy_logsumexp():
+    """window = grid, shift 0, nothing else: lse_i = logsumexp_j(q_i . k_j / sqrt(d))."""
+    from scipy.special import logsumexp
+
+    geo = O.Geometry(grid=(2, 4, 6), window=(2, 4, 6))
+    q, k, v = _qkv(geo, B=1, h=2, d=16, seed=17)
+    q *= 3.0  # spread the scores so the max term matters
+    _, lse = O.branch_attention(q, k, v, geo, O.KEYS_ALL)
+    for hh in range(2):
+        ref = logsumexp(q[0, hh] @ k[0, hh].T / 4.0, axis=1)
+        np.testing.assert_allclose(lse[0, hh], ref, rtol=0, atol=1e-12)

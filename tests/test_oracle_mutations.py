@@ -32,6 +32,9 @@ MUTATIONS = [
     ("scale", "scale = 1.0 / np.sqrt(d)", "scale = 1.0 / d", ["closed_form"]),
     ("softmax axis", "s = s - s.max(axis=1, keepdims=True)\n                p = np.exp(s)\n                p = p / p.sum(axis=1, keepdims=True)\n                Ow", "s = s - s.max(axis=0, keepdims=True)\n                p = np.exp(s)\n                p = p / p.sum(axis=0, keepdims=True)\n                Ow", ["closed_form", "rows_sum"]),
     ("routed window id", "u = int(route_idx[b, hh, w, r])", "u = int(route_idx[b, hh, (w + 1) % geo.n_win, r])", ["dense_masked"]),
+    ("lse drops the max", "Lw[b, hh, w] = (m + np.log(l))[:, 0]", "Lw[b, hh, w] = np.log(l)[:, 0]", ["lse_scipy", "branch_merge"]),
+    ("merge unnormalised", "out = sum(wts[i][..., None] * np.asarray(outs[i], dtype=np.float64) for i in range(len(outs))) / tot[..., None]", "out = sum(wts[i][..., None] * np.asarray(outs[i], dtype=np.float64) for i in range(len(outs)))", ["branch_merge"]),
+    ("branch drops routed", "for u in [w] + [int(route_idx[b, hh, w, r]) for r in range(geo.routed_k)]:", "for u in [w]:", ["branch_merge", "lse_zero_q"]),
     ("unshift output", "O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)", "O = window_unpartition(Ow, geo.grid, geo.window)", ["dense_masked"]),
 ]
 
@@ -51,6 +54,9 @@ PINS = {
     "constant_scores": lambda: [pins.test_constant_scores_give_mean_of_key_values(g) for g in pins.TINY_GEOS],
     "closed_form": lambda: pins.test_closed_form_whole_grid_is_dense_sdpa(),
     "rows_sum": lambda: [pins.test_softmax_rows_sum_to_one(g) for g in pins.TINY_GEOS],
+    "lse_scipy": lambda: pins.test_lse_whole_grid_is_scipy_logsumexp(),
+    "lse_zero_q": lambda: pins.test_lse_of_zero_queries_is_log_of_key_count(),
+    "branch_merge": lambda: [pins.test_branches_merge_to_the_joint_softmax(g) for g in pins.TINY_GEOS],
 }
 
 
