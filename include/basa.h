@@ -160,6 +160,13 @@ basa_status basa_pool_route(const void *q, const void *k, const void *v,
                             float *route_score, void *workspace,
                             const basa_params *p, basa_stream_t stream);
 
+/* Key groups of the branch form (basa_window_attn_fwd_lse). */
+#define BASA_KEYS_WINDOWS 1u /* the query's own window and its routed windows */
+#define BASA_KEYS_POOLED 2u  /* the pooled tokens kp, vp */
+#define BASA_KEYS_TEXT 4u    /* the n_text text rows of k, v */
+#define BASA_KEYS_ALL 7u
+#define BASA_MAX_BRANCHES 4
+
 /*
  * basa_window_attn_fwd — shifted-window attention forward (BASA §3.1 shifted
  * windows; §A.1: the local and global/text branches equal ONE softmax over the
@@ -180,6 +187,43 @@ basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v,
                                  const void *kp, const void *vp,
                                  const int32_t *route_idx, void *out,
                                  const basa_params *p, basa_stream_t stream);
+
+/*
+ * basa_window_attn_fwd_lse — one branch of the decomposed form (BASA §A.1: the
+ * local-window and text/global-memory branches can be evaluated separately and
+ * remain equivalent to one softmax over the concatenated K/V).
+ *
+ * As basa_window_attn_fwd, with the key list restricted to the groups in `keys`
+ * (an OR of BASA_KEYS_*; a group the layer does not have, pooled keys without a
+ * pool patch or text keys with n_text == 0, adds no keys, and a selection that
+ * leaves no key at all is BASA_ERR_INVALID_ARG),
+ * and, when `lse` is not NULL, the log-sum-exp of each query's scaled scores:
+ *   lse[b,h,i] = log sum_j exp(q_i . k_j / sqrt(head_dim))   (natural log)
+ * over the selected keys, float32 [B, heads, N] at original token positions
+ * (device, 4-byte aligned). keys = BASA_KEYS_ALL with lse = NULL is exactly
+ * basa_window_attn_fwd. Pointer rules for kp, vp, route_idx are those of
+ * basa_window_attn_fwd (pass them whenever the layer has them).
+ */
+basa_status basa_window_attn_fwd_lse(const void *q, const void *k, const void *v,
+                                     const void *kp, const void *vp,
+                                     const int32_t *route_idx, void *out, float *lse,
+                                     uint32_t keys, const basa_params *p,
+                                     basa_stream_t stream);
+
+/*
+ * basa_merge_branches — joint softmax from n branch results (BASA §A.1).
+ *
+ *   L[r]   = log sum_b exp(lses[b][r])
+ *   out[r] = sum_b exp(lses[b][r] - L[r]) * outs[b][r]      (float32 arithmetic)
+ * for every query row r of [B, heads, N]; `lse` (nullable) receives L. `outs`
+ * and `lses` are HOST arrays of n (1 <= n <= BASA_MAX_BRANCHES) DEVICE pointers:
+ * outs[b] like `out` of basa_window_attn_fwd (element type p->dtype, 16-byte
+ * aligned), lses[b] float32 [B, heads, N]. `out` may alias outs[0] (each
+ * element is read before it is written by the same thread).
+ */
+basa_status basa_merge_branches(int n, const void *const *outs, const float *const *lses,
+                                void *out, float *lse, const basa_params *p,
+                                basa_stream_t stream);
 
 /*
  * basa_route_windows_noalloc — basa_route_windows without a caller workspace.

@@ -25,6 +25,8 @@ STATUS_NAMES = {
 BASA_BF16 = 0
 BASA_F32 = 1
 BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD = 0x1
+BASA_KEYS_WINDOWS, BASA_KEYS_POOLED, BASA_KEYS_TEXT, BASA_KEYS_ALL = 1, 2, 4, 7
+BASA_MAX_BRANCHES = 4
 EXPORTED = (
     "basa_pool_kv",
     "basa_route_workspace_bytes",
@@ -33,6 +35,8 @@ EXPORTED = (
     "basa_pool_route_workspace_bytes",
     "basa_pool_route",
     "basa_window_attn_fwd",
+    "basa_window_attn_fwd_lse",
+    "basa_merge_branches",
     "basa_status_string",
     "basa_device_error_status",
 )
@@ -80,6 +84,10 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.basa_pool_route.restype = ctypes.c_int
     lib.basa_window_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, P, vp]
     lib.basa_window_attn_fwd.restype = ctypes.c_int
+    lib.basa_window_attn_fwd_lse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32, P, vp]
+    lib.basa_window_attn_fwd_lse.restype = ctypes.c_int
+    lib.basa_merge_branches.argtypes = [ctypes.c_int, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp, P, vp]
+    lib.basa_merge_branches.restype = ctypes.c_int
     lib.basa_status_string.argtypes = [ctypes.c_int]
     lib.basa_status_string.restype = ctypes.c_char_p
     lib.basa_device_error_status.argtypes = [ctypes.c_int32]
@@ -183,4 +191,23 @@ def basa_window_attn_fwd(q, k, v, kp, vp, route_idx, out, params: basa_params, s
                                    ctypes.byref(params), _stream(stream))
     if check:
         _check(st, "basa_window_attn_fwd")
+    return st
+
+
+def basa_window_attn_fwd_lse(q, k, v, kp, vp, route_idx, out, lse, keys: int, params: basa_params, stream=None,
+                             check=True) -> int:
+    st = _lib.basa_window_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp), _ptr(route_idx), _ptr(out),
+                                       _ptr(lse), keys, ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_window_attn_fwd_lse")
+    return st
+
+
+def basa_merge_branches(outs, lses, out, lse, params: basa_params, stream=None, check=True) -> int:
+    n = len(outs)
+    arr_o = (ctypes.c_void_p * max(n, 1))(*[_ptr(x) for x in outs])
+    arr_l = (ctypes.c_void_p * max(n, 1))(*[_ptr(x) for x in lses])
+    st = _lib.basa_merge_branches(n, arr_o, arr_l, _ptr(out), _ptr(lse), ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_merge_branches")
     return st

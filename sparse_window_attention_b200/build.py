@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbasa.so")
-SOURCES = ["api.cpp", "plan.cpp", "pool_route.cu", "pool_route_fused.cu", "attn_f32.cu", "attn_bf16_sm100.cu"]
+SOURCES = ["api.cpp", "plan.cpp", "pool_route.cu", "pool_route_fused.cu", "merge.cu", "attn_f32.cu", "attn_bf16_sm100.cu"]
 HEADERS = [os.path.join(CSRC, h) for h in ("basa_internal.h", "sm100_ptx.cuh")] + [os.path.join(ROOT, "include", "basa.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -146,12 +146,17 @@ basa_status basa_pool_route(const void *q, const void *k, const void *v, void *k
                                        reinterpret_cast<cudaStream_t>(stream));
 }
 
-basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
-                                 const int32_t *route_idx, void *out, const basa_params *p,
-                                 basa_stream_t stream) {
+static basa_status attn_common(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                               const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params *p,
+                               basa_stream_t stream) {
   basa_status st = check_common(p);
   if (st != BASA_OK) return st;
   if (p->dtype == BASA_BF16 && p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (keys & ~BASA_KEYS_ALL) return BASA_ERR_INVALID_ARG;
+  // groups the layer does not have add no keys; the selection must leave some
+  const bool any = (keys & BASA_KEYS_WINDOWS) || ((keys & BASA_KEYS_POOLED) && has_pool(p)) ||
+                   ((keys & BASA_KEYS_TEXT) && p->n_text > 0);
+  if (!any) return BASA_ERR_INVALID_ARG;
   if (empty_batch(p)) return BASA_OK;
   if (!q || !k || !v || !out) return BASA_ERR_INVALID_ARG;
   if (has_pool(p) != (kp != nullptr) || has_pool(p) != (vp != nullptr)) return BASA_ERR_INVALID_ARG;
@@ -159,9 +164,35 @@ basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, co
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return BASA_ERR_INVALID_ARG;
   if (kp && (!aligned16(kp) || !aligned16(vp))) return BASA_ERR_INVALID_ARG;
   if (route_idx && !aligned4(route_idx)) return BASA_ERR_INVALID_ARG;
+  if (lse && !aligned4(lse)) return BASA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (p->dtype == BASA_F32) return basa::launch_attn_f32(q, k, v, kp, vp, route_idx, out, *p, s);
-  return basa::launch_attn_bf16(q, k, v, kp, vp, route_idx, out, *p, s);
+  if (p->dtype == BASA_F32) return basa::launch_attn_f32(q, k, v, kp, vp, route_idx, out, lse, keys, *p, s);
+  return basa::launch_attn_bf16(q, k, v, kp, vp, route_idx, out, lse, keys, *p, s);
+}
+
+basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                                 const int32_t *route_idx, void *out, const basa_params *p,
+                                 basa_stream_t stream) {
+  return attn_common(q, k, v, kp, vp, route_idx, out, nullptr, BASA_KEYS_ALL, p, stream);
+}
+
+basa_status basa_window_attn_fwd_lse(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                                     const int32_t *route_idx, void *out, float *lse, uint32_t keys,
+                                     const basa_params *p, basa_stream_t stream) {
+  return attn_common(q, k, v, kp, vp, route_idx, out, lse, keys, p, stream);
+}
+
+basa_status basa_merge_branches(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
+                                const basa_params *p, basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (n < 1 || n > BASA_MAX_BRANCHES) return BASA_ERR_INVALID_ARG;
+  if (empty_batch(p)) return BASA_OK;
+  if (!outs || !lses || !out || !aligned16(out)) return BASA_ERR_INVALID_ARG;
+  if (lse && !aligned4(lse)) return BASA_ERR_INVALID_ARG;
+  for (int b = 0; b < n; ++b)
+    if (!outs[b] || !lses[b] || !aligned16(outs[b]) || !aligned4(lses[b])) return BASA_ERR_INVALID_ARG;
+  return basa::launch_merge(n, outs, lses, out, lse, *p, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

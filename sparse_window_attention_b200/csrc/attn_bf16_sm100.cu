@@ -66,6 +66,8 @@ struct alignas(64) AttnParams {
   Geo g;
   int routed_k, n_pool, n_text, n_pool_tiles, n_text_tiles;
   float scale_log2;
+  int use_windows;  // own and routed windows are keys (else pooled and/or text only)
+  float *lse;       // nullable: log-sum-exp of each query row's scaled scores [B*heads][N]
   int all_full;  // every key tile of the launch is full: no column masks
   uint32_t flags;
   unsigned long long timeout_ns;
@@ -116,7 +118,7 @@ struct KeyIter {
 };
 
 __device__ __forceinline__ int seg_tiles(const AttnParams &P, const Ctrl &c, int seg) {
-  if (seg <= P.routed_k) return P.plan.type[c.wtype[seg]].n_tiles;
+  if (seg <= P.routed_k) return P.use_windows ? P.plan.type[c.wtype[seg]].n_tiles : 0;
   if (seg == P.routed_k + 1) return P.n_pool_tiles;
   return P.n_text_tiles;
 }
@@ -126,6 +128,13 @@ __device__ __forceinline__ void advance(const AttnParams &P, const Ctrl &c, KeyI
     ++it.seg;
     it.t = 0;
   }
+}
+
+// First key tile of the stream (segments without tiles are skipped).
+__device__ __forceinline__ KeyIter first_key(const AttnParams &P, const Ctrl &c) {
+  KeyIter it{0, 0};
+  while (it.seg <= P.routed_k + 2 && seg_tiles(P, c, it.seg) == 0) ++it.seg;
+  return it;
 }
 
 __device__ __forceinline__ int wrap(int x, int g) { return x >= g ? x - g : x; }
@@ -360,8 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
   ptx::tc_fence_after();
   const uint32_t tmem = c.tmem_base;
 
-  int n_kt = P.n_pool_tiles + P.n_text_tiles;
-  for (int s = 0; s <= P.routed_k; ++s) n_kt += P.plan.type[c.wtype[s]].n_tiles;
+  int n_kt = 0;
+  for (int s = 0; s <= P.routed_k + 2; ++s) n_kt += seg_tiles(P, c, s);
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA loader
@@ -375,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       for (int g = 0; g < (has_q1 ? 2 : 1); ++g)
         load_window_tile(P, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh, smem + kSmemQ + g * kTileBytes,
                          &c.q_full);
-      KeyIter it{0, 0};
+      KeyIter it = first_key(P, c);
       int last = -1;
       bool skipped0 = false;
       for (int j = 0; j < n_kt; ++j) {
@@ -494,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     }
     float m = -INFINITY, l = 0.f;
     bool ok = active;
-    KeyIter it{0, 0};
+    KeyIter it = first_key(P, c);
     for (int j = 0; ok && j < n_kt; ++j) {
       ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.s_full[g], j & 1));
       if (!ok) break;
@@ -581,6 +590,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       }
       ptx::fence_proxy_async_smem();
     }
+    if (ok && P.lse != nullptr) {
+      // log-sum-exp of this row: m and l are in base 2 of the scaled scores
+      const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
+      for (int i = 0; i < tile.n_pieces; ++i) {
+        const PlanPiece pc = P.plan.piece[tile.first_piece + i];
+        const PlanShape sh = P.plan.shape[pc.shape];
+        const int local = row - int(pc.dest);
+        if (local < 0 || local >= sh.rows) continue;
+        const int lx = local % sh.cx, ly = (local / sh.cx) % sh.cy, lt = local / (sh.cx * sh.cy);
+        const int x = wrap(ox + pc.lx, P.g.W) + lx, y = wrap(oy + pc.ly, P.g.H) + ly, t = wrap(ot + pc.lt, P.g.T) + lt;
+        P.lse[(long long)bh * P.g.N + ((long long)t * P.g.H + y) * P.g.W + x] = (m + log2f(l)) * 0.6931471805599453f;
+      }
+    }
     ptx::named_barrier(1 + g, 128);
     if (active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
       const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
@@ -650,7 +672,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
-                             const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s) {
+                             const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params &p,
+                             cudaStream_t s) {
   if (!encode_fn()) return BASA_ERR_CUDA;
   AttnParams P;
   std::memset(&P, 0, sizeof(P));
@@ -675,8 +698,10 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
   if (p.n_text > 0) {
     if (!encode_rows_map(&P.map_kt, k, p, kv_rows) || !encode_rows_map(&P.map_vt, v, p, kv_rows)) return BASA_ERR_CUDA;
   }
-  P.n_pool_tiles = (P.n_pool + kTileRows - 1) / kTileRows;
-  P.n_text_tiles = (p.n_text + kTileRows - 1) / kTileRows;
+  P.n_pool_tiles = (keys & BASA_KEYS_POOLED) ? (P.n_pool + kTileRows - 1) / kTileRows : 0;
+  P.n_text_tiles = (keys & BASA_KEYS_TEXT) ? (p.n_text + kTileRows - 1) / kTileRows : 0;
+  P.use_windows = (keys & BASA_KEYS_WINDOWS) ? 1 : 0;
+  P.lse = lse;
   P.route = route_idx;
   P.dev_err = p.dev_err;
   P.routed_k = p.routed_k;

@@ -17,15 +17,18 @@ struct F32Args {
   const float *q, *k, *v, *kp, *vp;
   const int32_t *route;
   float *out;
+  float *lse;  // nullable [B*heads][N]
   Geo g;
   int heads, d, n_text, n_pool, routed_k, win_tok, q_chunks;
+  int n_vis_keys, n_pool_keys, n_text_keys;  // keys taken from each group (0 = group not selected)
   float scale;
 };
 
-// Row of key j of window w's key list: [own | routed windows | pooled | text].
+// Row of key j of window w's key list: [own | routed windows | pooled | text],
+// restricted to the selected groups.
 __device__ __forceinline__ const float *key_row(const F32Args &a, const float *kv, const float *kvp, long long bh,
                                                 const int *wins, int j) {
-  const int nvis = a.win_tok * (1 + a.routed_k);
+  const int nvis = a.n_vis_keys;
   const long long rows = (long long)a.g.N + a.n_text;
   if (j < nvis) {
     const int u = wins[j / a.win_tok];
@@ -37,8 +40,8 @@ __device__ __forceinline__ const float *key_row(const F32Args &a, const float *k
     return kv + (bh * rows + ((long long)t * a.g.H + y) * a.g.W + x) * a.d;
   }
   j -= nvis;
-  if (j < a.n_pool) return kvp + (bh * a.n_pool + j) * a.d;
-  j -= a.n_pool;
+  if (j < a.n_pool_keys) return kvp + (bh * a.n_pool + j) * a.d;
+  j -= a.n_pool_keys;
   return kv + (bh * rows + a.g.N + j) * a.d;
 }
 
@@ -76,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(F32Args a) {
     o[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int nk = a.win_tok * (1 + a.routed_k) + a.n_pool + a.n_text;
+  const int nk = a.n_vis_keys + a.n_pool_keys + a.n_text_keys;
   for (int k0 = 0; k0 < nk; k0 += kKeyTile) {
     __syncthreads();
     for (int i = threadIdx.x; i < kKeyTile * (D / 4); i += kThreads) {
@@ -120,13 +123,15 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(F32Args a) {
     float *op = a.out + (bh * a.g.N + qtok) * D;
 #pragma unroll
     for (int i = 0; i < 64; ++i) op[i * TPQ + half] = o[i] * inv;
+    if (a.lse && half == 0) a.lse[bh * a.g.N + qtok] = m + logf(l);
   }
 }
 
 }  // namespace
 
 basa_status launch_attn_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
-                            const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s) {
+                            const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params &p,
+                            cudaStream_t s) {
   F32Args a{};
   a.q = static_cast<const float *>(q);
   a.k = static_cast<const float *>(k);
@@ -142,6 +147,10 @@ basa_status launch_attn_f32(const void *q, const void *k, const void *v, const v
   a.n_pool = p.pt > 0 ? (p.T / p.pt) * (p.H / p.ph) * (p.W / p.pw) : 0;
   a.routed_k = p.routed_k;
   a.win_tok = p.wt * p.wh * p.ww;
+  a.lse = lse;
+  a.n_vis_keys = (keys & BASA_KEYS_WINDOWS) ? a.win_tok * (1 + a.routed_k) : 0;
+  a.n_pool_keys = (keys & BASA_KEYS_POOLED) ? a.n_pool : 0;
+  a.n_text_keys = (keys & BASA_KEYS_TEXT) ? a.n_text : 0;
   const int qpb = kThreads / (p.head_dim / 64);
   a.q_chunks = (a.win_tok + qpb - 1) / qpb;
   a.scale = 1.0f / sqrtf(float(p.head_dim));

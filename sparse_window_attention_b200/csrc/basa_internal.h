@@ -132,9 +132,16 @@ basa_status launch_topk(const float *qm, const float *km, int32_t *route_idx, fl
 // Fused pooling + window means + top-k; `workspace` holds means_bytes + part_bytes.
 basa_status launch_pool_route_fused(const void *q, const void *k, const void *v, void *kp, void *vp, int32_t *route_idx,
                                     float *route_score, void *workspace, const basa_params &p, cudaStream_t s);
+// `lse` (nullable) receives each query's log-sum-exp; `keys` selects key groups
+// (BASA_KEYS_* bits).
 basa_status launch_attn_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
-                            const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
+                            const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params &p,
+                            cudaStream_t s);
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
-                             const int32_t *route_idx, void *out, const basa_params &p, cudaStream_t s);
+                             const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params &p,
+                             cudaStream_t s);
+// out = sum_b exp(lse_b - L) out_b, L = log sum_b exp(lse_b), over n branches.
+basa_status launch_merge(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
+                         const basa_params &p, cudaStream_t s);
 
 }  // namespace basa

@@ -74,6 +74,39 @@ class BasaLayer:
         route_idx = self.route_idx if route_idx is None else route_idx
         B.basa_window_attn_fwd(q, k, v, kp, vp, route_idx, out, self.params(shift, **extra), stream)
 
+    def attention_lse(self, q, k, v, out, lse, shift, keys, kp=None, vp=None, route_idx=None, stream=None):
+        """One branch: attention over the key groups in ``keys`` and its log-sum-exp."""
+        kp = self.kp if kp is None else kp
+        vp = self.vp if vp is None else vp
+        route_idx = self.route_idx if route_idx is None else route_idx
+        B.basa_window_attn_fwd_lse(q, k, v, kp, vp, route_idx, out, lse, keys, self.params(shift), stream)
+
+    def merge(self, outs, lses, out, lse=None, stream=None):
+        """Joint softmax from branch results (basa_merge_branches)."""
+        B.basa_merge_branches(outs, lses, out, lse, self.params((0, 0, 0)), stream)
+
+    def forward_branches(self, q, k, v, shift, splits, out=None, stream=None):
+        """The layer in branch form: pooled K/V and routing as in forward(), then one
+        attention call per key-group set in ``splits`` (e.g. [WINDOWS, POOLED | TEXT])
+        and their merge."""
+        if out is None:
+            out = torch.empty_like(q)
+        if self.fused and self.fused_bytes(shift) > 0:
+            self.pool_route(q, k, v, shift, stream)
+        else:
+            if self.has_pool:
+                self.pool_kv(k, v, shift, stream)
+            if self.routed_k > 0:
+                self.route(q, k, shift, stream)
+        if not hasattr(self, "_branch_bufs") or len(self._branch_bufs) < len(splits):
+            self._branch_bufs = [(torch.empty_like(q), torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device))
+                                 for _ in splits]
+        for (o, l), keys in zip(self._branch_bufs, splits):
+            self.attention_lse(q, k, v, o, l, shift, keys, stream=stream)
+        bufs = self._branch_bufs[: len(splits)]
+        self.merge([o for o, _ in bufs], [l for _, l in bufs], out, None, stream)
+        return out
+
     def forward(self, q, k, v, shift, out=None, stream=None):
         """Full layer: pooled K/V, routed windows (if routed_k > 0), attention."""
         if out is None:

@@ -141,6 +141,25 @@ def test_fused_pool_route_checks():
     assert B.basa_pool_route_workspace_bytes(p) > 2 * 12 * 16 * 128 * 4
 
 
+def test_branch_form_checks():
+    p = _p()  # pool and 16 text rows, no routing
+    call = lambda keys, pp=p: B.basa_window_attn_fwd_lse(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, keys, pp,
+                                                         stream=0, check=False)
+    assert call(0) == 1 and call(8) == 1
+    nop = _p(pool=(0, 0, 0))
+    assert B.basa_window_attn_fwd_lse(FAKE, FAKE, FAKE, None, None, None, FAKE, None, B.BASA_KEYS_POOLED, nop,
+                                      stream=0, check=False) == 1
+    assert call(B.BASA_KEYS_TEXT, _p(n_text=0)) == 1
+    assert B.basa_window_attn_fwd_lse(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE + 2, B.BASA_KEYS_ALL, p,
+                                      stream=0, check=False) == 1  # misaligned lse
+    merge = lambda outs, lses, out=FAKE: B.basa_merge_branches(outs, lses, out, None, p, stream=0, check=False)
+    assert merge([], []) == 1
+    assert merge([FAKE] * 5, [FAKE] * 5) == 1
+    assert merge([FAKE, None], [FAKE, FAKE]) == 1
+    assert merge([FAKE, FAKE + 8], [FAKE, FAKE]) == 1
+    assert merge([FAKE], [FAKE], out=None) == 1
+
+
 def test_route_workspace_bytes():
     p = _p(routed_k=2)
     assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4
