@@ -262,10 +262,40 @@ def run_ours(args, world, rank, local):
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world)
     if not args.no_extra and world == 1:
+        res["branch_form"] = run_branch_form(args, layer, qd, kd, vd, shifts, flops)
         for name in ("wan", "wan_video"):
             if args.workload != name:
                 res["also_" + name] = run_also(args, name)
     return res
+
+
+def run_branch_form(args, layer, qd, kd, vd, shifts, flops):
+    """The same layer in the branch form (BASA §A.1): local windows and the pooled +
+    text keys as two attention calls with log-sum-exp, then their merge. Context
+    for the single-pass kernel, which needs neither the second pass over Q nor the
+    merge."""
+    from sparse_window_attention_b200 import binding as B
+
+    groups = (B.BASA_KEYS_POOLED if layer.has_pool else 0) | (B.BASA_KEYS_TEXT if layer.n_text else 0)
+    if not groups:
+        return None
+    splits = [B.BASA_KEYS_WINDOWS, groups]
+    out = torch.empty_like(qd)
+    steps = max(10, args.steps // 10)
+    for i in range(3):
+        layer.forward_branches(qd, kd, vd, shifts[i % len(shifts)], splits, out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        layer.forward_branches(qd, kd, vd, shifts[i % len(shifts)], splits, out=out)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    return {"splits": "windows | pooled + text", "ms_per_step": round(ms, 4),
+            "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "launches_per_step": layer.launches_per_forward() + len(splits)}
 
 
 def hbm_lines(cnt, pool_ms, route_ms, hbm_gbs, fused):

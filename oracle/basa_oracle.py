@@ -343,6 +343,30 @@ def merge_branches(outs, lses):
     return out, m + np.log(tot)
 
 
+def text_query_attention(q_text, k, v, geo: Geometry):
+    """Output rows of the text queries: dense attention over every key.
+
+    The pages sparsify the image queries' keys only; a text query keeps the dense
+    model's joint attention over all N visual keys and the n_text text keys (the
+    text/global-memory branch of BASA §A.1 seen from the text side). out[i] =
+    sum_j softmax_j(q_i . k_j / sqrt(d)) v_j over the N + n_text rows of k, v.
+    q_text [B, h, n_text, d] -> [B, h, n_text, d] float64.
+    """
+    qt = np.asarray(q_text, dtype=np.float64)
+    k64 = np.asarray(k, dtype=np.float64)
+    v64 = np.asarray(v, dtype=np.float64)
+    B, h, nt, d = qt.shape
+    assert k64.shape[2] == geo.N + geo.n_text and nt == geo.n_text
+    out = np.empty_like(qt)
+    for b in range(B):
+        for hh in range(h):
+            s = (qt[b, hh] @ k64[b, hh].T) / np.sqrt(d)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            out[b, hh] = (p / p.sum(axis=1, keepdims=True)) @ v64[b, hh]
+    return out
+
+
 def window_of_token(geo: Geometry):
     """Window id of every token of the ORIGINAL grid, computed without any roll.
 

@@ -473,3 +473,29 @@ def test_lse_whole_grid_is_scipy_logsumexp():
     for hh in range(2):
         ref = logsumexp(q[0, hh] @ k[0, hh].T / 4.0, axis=1)
         np.testing.assert_allclose(lse[0, hh], ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- text-query rows
+
+
+def test_text_queries_dense_sdpa():
+    """Text queries attend to every visual and text key: torch SDPA in float64
+    over the concatenated rows."""
+    geo = O.Geometry(grid=(2, 4, 6), window=(1, 2, 3), shift=(1, 1, 2), pool=(1, 2, 3), n_text=5, routed_k=1)
+    rng = np.random.default_rng(31)
+    qt = rng.standard_normal((2, 3, 5, 16))
+    k = rng.standard_normal((2, 3, geo.N + 5, 16))
+    v = rng.standard_normal((2, 3, geo.N + 5, 16))
+    out = O.text_query_attention(qt, k, v, geo)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(qt), torch.from_numpy(k),
+                                                           torch.from_numpy(v)).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_text_queries_zero_query_is_mean_of_all_values():
+    geo = O.Geometry(grid=(1, 4, 4), window=(1, 2, 2), n_text=3)
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((1, 2, geo.N + 3, 8))
+    v = rng.standard_normal((1, 2, geo.N + 3, 8))
+    out = O.text_query_attention(np.zeros((1, 2, 3, 8)), k, v, geo)
+    np.testing.assert_allclose(out, np.broadcast_to(v.mean(axis=2, keepdims=True), out.shape), rtol=0, atol=1e-12)

@@ -35,6 +35,8 @@ MUTATIONS = [
     ("lse drops the max", "Lw[b, hh, w] = (m + np.log(l))[:, 0]", "Lw[b, hh, w] = np.log(l)[:, 0]", ["lse_scipy", "branch_merge"]),
     ("merge unnormalised", "out = sum(wts[i][..., None] * np.asarray(outs[i], dtype=np.float64) for i in range(len(outs))) / tot[..., None]", "out = sum(wts[i][..., None] * np.asarray(outs[i], dtype=np.float64) for i in range(len(outs)))", ["branch_merge"]),
     ("branch drops routed", "for u in [w] + [int(route_idx[b, hh, w, r]) for r in range(geo.routed_k)]:", "for u in [w]:", ["branch_merge", "lse_zero_q"]),
+    ("text queries skip text keys", "            s = (qt[b, hh] @ k64[b, hh].T) / np.sqrt(d)", "            s = (qt[b, hh] @ k64[b, hh, : geo.N].T) / np.sqrt(d)", ["text_sdpa", "text_zero_q"]),
+    ("text queries scale", "            s = (qt[b, hh] @ k64[b, hh].T) / np.sqrt(d)", "            s = (qt[b, hh] @ k64[b, hh].T) / d", ["text_sdpa"]),
     ("unshift output", "O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)", "O = window_unpartition(Ow, geo.grid, geo.window)", ["dense_masked"]),
 ]
 
@@ -55,6 +57,8 @@ PINS = {
     "closed_form": lambda: pins.test_closed_form_whole_grid_is_dense_sdpa(),
     "rows_sum": lambda: [pins.test_softmax_rows_sum_to_one(g) for g in pins.TINY_GEOS],
     "lse_scipy": lambda: pins.test_lse_whole_grid_is_scipy_logsumexp(),
+    "text_sdpa": lambda: pins.test_text_queries_dense_sdpa(),
+    "text_zero_q": lambda: pins.test_text_queries_zero_query_is_mean_of_all_values(),
     "lse_zero_q": lambda: pins.test_lse_of_zero_queries_is_log_of_key_count(),
     "branch_merge": lambda: [pins.test_branches_merge_to_the_joint_softmax(g) for g in pins.TINY_GEOS],
 }
