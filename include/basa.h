@@ -211,6 +211,23 @@ basa_status basa_window_attn_fwd_lse(const void *q, const void *k, const void *v
                                      basa_stream_t stream);
 
 /*
+ * basa_text_attn_fwd — output rows of the text queries. The pages sparsify the
+ * image queries only; a text query keeps dense joint attention over every key
+ * (the N visual rows and the n_text text rows of k, v; BASA §A.1's text branch
+ * seen from the text side):
+ *   out_text[b,h,i] = sum_j softmax_j(q_text[b,h,i] . k[b,h,j] / sqrt(head_dim)) v[b,h,j]
+ * q_text, out_text: [B, heads, n_text, head_dim] (device, 16-byte aligned);
+ * k, v as for basa_window_attn_fwd. Requires n_text >= 1. `workspace` (device,
+ * 16-byte aligned, contents ignored) holds basa_text_attn_workspace_bytes(p)
+ * bytes of per-split partial results (0 bytes: pass NULL): with bfloat16 the key
+ * range is split over CTAs and the splits are merged by their log-sum-exp.
+ */
+size_t basa_text_attn_workspace_bytes(const basa_params *p);
+basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v,
+                               void *out_text, void *workspace, const basa_params *p,
+                               basa_stream_t stream);
+
+/*
  * basa_merge_branches — joint softmax from n branch results (BASA §A.1).
  *
  *   L[r]   = log sum_b exp(lses[b][r])

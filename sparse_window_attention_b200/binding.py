@@ -37,6 +37,8 @@ EXPORTED = (
     "basa_window_attn_fwd",
     "basa_window_attn_fwd_lse",
     "basa_merge_branches",
+    "basa_text_attn_workspace_bytes",
+    "basa_text_attn_fwd",
     "basa_status_string",
     "basa_device_error_status",
 )
@@ -88,6 +90,10 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.basa_window_attn_fwd_lse.restype = ctypes.c_int
     lib.basa_merge_branches.argtypes = [ctypes.c_int, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp, P, vp]
     lib.basa_merge_branches.restype = ctypes.c_int
+    lib.basa_text_attn_workspace_bytes.argtypes = [P]
+    lib.basa_text_attn_workspace_bytes.restype = ctypes.c_size_t
+    lib.basa_text_attn_fwd.argtypes = [vp, vp, vp, vp, vp, P, vp]
+    lib.basa_text_attn_fwd.restype = ctypes.c_int
     lib.basa_status_string.argtypes = [ctypes.c_int]
     lib.basa_status_string.restype = ctypes.c_char_p
     lib.basa_device_error_status.argtypes = [ctypes.c_int32]
@@ -210,4 +216,16 @@ def basa_merge_branches(outs, lses, out, lse, params: basa_params, stream=None, 
     st = _lib.basa_merge_branches(n, arr_o, arr_l, _ptr(out), _ptr(lse), ctypes.byref(params), _stream(stream))
     if check:
         _check(st, "basa_merge_branches")
+    return st
+
+
+def basa_text_attn_workspace_bytes(params: basa_params) -> int:
+    return _lib.basa_text_attn_workspace_bytes(ctypes.byref(params))
+
+
+def basa_text_attn_fwd(q_text, k, v, out_text, workspace, params: basa_params, stream=None, check=True) -> int:
+    st = _lib.basa_text_attn_fwd(_ptr(q_text), _ptr(k), _ptr(v), _ptr(out_text), _ptr(workspace),
+                                 ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_text_attn_fwd")
     return st

@@ -182,6 +182,28 @@ basa_status basa_window_attn_fwd_lse(const void *q, const void *k, const void *v
   return attn_common(q, k, v, kp, vp, route_idx, out, lse, keys, p, stream);
 }
 
+size_t basa_text_attn_workspace_bytes(const basa_params *p) {
+  if (check_common(p) != BASA_OK || p->n_text < 1 || p->dtype != BASA_BF16) return 0;
+  return basa::text_attn_workspace(*p, basa::device_sm_count());
+}
+
+basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v, void *out_text, void *workspace,
+                               const basa_params *p, basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (p->n_text < 1) return BASA_ERR_INVALID_ARG;
+  if (p->dtype == BASA_BF16 && p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q_text || !k || !v || !out_text) return BASA_ERR_INVALID_ARG;
+  if (!aligned16(q_text) || !aligned16(k) || !aligned16(v) || !aligned16(out_text)) return BASA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == BASA_F32) return basa::launch_attn_text_f32(q_text, k, v, out_text, *p, s);
+  const int sms = basa::device_sm_count();
+  if (sms <= 0) return BASA_ERR_CUDA;
+  if (basa::text_attn_workspace(*p, sms) > 0 && (!workspace || !aligned16(workspace))) return BASA_ERR_INVALID_ARG;
+  return basa::launch_attn_text_bf16(q_text, k, v, out_text, workspace, *p, sms, s);
+}
+
 basa_status basa_merge_branches(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
                                 const basa_params *p, basa_stream_t stream) {
   basa_status st = check_common(p);

@@ -45,7 +45,8 @@ constexpr int kMaskTable = 64;                         // key tiles whose column
 constexpr uint32_t kSmemMask = kSmemCtrl + kCtrlBytes;
 constexpr uint32_t kSmemBytes = kSmemMask + kMaskTable * 16 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr int kDefaultEmuPairs = 0;  // exponential pairs of every 8 done on the FMA pipe
+constexpr int kDefaultEmuPairs = 0;
+constexpr int kMaxTextSplits = 8;  // key-range splits of the text-query rows  // exponential pairs of every 8 done on the FMA pipe
 
 // tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), N >> 3 at bits 17-22, M >> 4 at bits 24-28; bit 16 marks
@@ -60,6 +61,7 @@ struct alignas(64) AttnParams {
   CUtensorMap map_v[kMaxShapes];
   CUtensorMap map_o[kMaxShapes];
   CUtensorMap map_kp, map_vp, map_kt, map_vt;
+  CUtensorMap map_qd, map_od;  // text-query mode: query rows and output rows (d, row, b*head)
   WindowPlan plan;
   const int32_t *route;
   int32_t *dev_err;
@@ -67,6 +69,11 @@ struct alignas(64) AttnParams {
   int routed_k, n_pool, n_text, n_pool_tiles, n_text_tiles;
   float scale_log2;
   int use_windows;  // own and routed windows are keys (else pooled and/or text only)
+  // Text-query mode: the queries are the n_text text rows and attend densely to
+  // every k/v row, which are streamed as the "text" segment starting at row 0.
+  // The key tiles are split into n_splits ranges, one per CTA group.
+  int dense, dense_rows, dense_q_tiles, dense_pairs, n_splits, split_tiles, bh_count;
+  int text_row0;  // first k/v row of the text segment: N (window mode) or 0
   float *lse;       // nullable: log-sum-exp of each query row's scaled scores [B*heads][N]
   int all_full;  // every key tile of the launch is full: no column masks
   uint32_t flags;
@@ -81,6 +88,7 @@ struct Ctrl {
   uint64_t q_full, s_full[2], p_full[2], o_full[2], drain;
   uint32_t tmem_base;
   int abort;
+  int tile0, ntile;  // text-query mode: this CTA's range of key tiles
   int wtype[1 + kMaxRouted];
   int org[1 + kMaxRouted][3];
 };
@@ -120,7 +128,7 @@ struct KeyIter {
 __device__ __forceinline__ int seg_tiles(const AttnParams &P, const Ctrl &c, int seg) {
   if (seg <= P.routed_k) return P.use_windows ? P.plan.type[c.wtype[seg]].n_tiles : 0;
   if (seg == P.routed_k + 1) return P.n_pool_tiles;
-  return P.n_text_tiles;
+  return P.dense ? c.ntile : P.n_text_tiles;
 }
 __device__ __forceinline__ void advance(const AttnParams &P, const Ctrl &c, KeyIter &it) {
   ++it.t;
@@ -163,7 +171,7 @@ __device__ __forceinline__ uint32_t load_key_tile(const AttnParams &P, const Ctr
   }
   const bool pooled = it.seg == P.routed_k + 1;
   const CUtensorMap *map = pooled ? (is_v ? &P.map_vp : &P.map_kp) : (is_v ? &P.map_vt : &P.map_kt);
-  const int row = (pooled ? 0 : P.g.N) + it.t * kTileRows;
+  const int row = pooled ? it.t * kTileRows : P.text_row0 + (c.tile0 + it.t) * kTileRows;
   ptx::tma_load_3d(dst, map, bar, 0, row, bh);
   ptx::tma_load_3d(dst + kHalfBytes, map, bar, 64, row, bh);
   return kTileBytes;
@@ -177,8 +185,9 @@ __device__ __forceinline__ bool key_tile_mask(const AttnParams &P, const Ctrl &c
     for (int i = 0; i < 4; ++i) m[i] = tile.mask[i];
     return tile.valid_rows == kTileRows;
   }
-  const int total = (it.seg == P.routed_k + 1) ? P.n_pool : P.n_text;
-  const int valid = min(kTileRows, total - it.t * kTileRows);
+  const bool pooled = it.seg == P.routed_k + 1;
+  const int total = pooled ? P.n_pool : (P.dense ? P.dense_rows : P.n_text);
+  const int valid = min(kTileRows, total - (pooled ? it.t : c.tile0 + it.t) * kTileRows);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int v = valid - 32 * i;
@@ -316,16 +325,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
   Ctrl &c = *reinterpret_cast<Ctrl *>(smem + kSmemCtrl);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  const int pairs = P.plan.max_pairs;
-  const int pair = blockIdx.x % pairs;
-  const int w = (blockIdx.x / pairs) % P.g.nWin;
-  const int bh = blockIdx.x / (pairs * P.g.nWin);
-  int ot, oy, ox, wtype;
-  window_origin(P.g, w, &ot, &oy, &ox, &wtype);
-  const PlanType ty = P.plan.type[wtype];
+  int pair, w = 0, bh, split = 0, ot = 0, oy = 0, ox = 0, wtype = 0, n_q_tiles;
+  PlanType ty{0, 0};
+  if (P.dense) {
+    pair = blockIdx.x % P.dense_pairs;
+    split = (blockIdx.x / P.dense_pairs) % P.n_splits;
+    bh = blockIdx.x / (P.dense_pairs * P.n_splits);
+    n_q_tiles = P.dense_q_tiles;
+  } else {
+    const int pairs = P.plan.max_pairs;
+    pair = blockIdx.x % pairs;
+    w = (blockIdx.x / pairs) % P.g.nWin;
+    bh = blockIdx.x / (pairs * P.g.nWin);
+    window_origin(P.g, w, &ot, &oy, &ox, &wtype);
+    ty = P.plan.type[wtype];
+    n_q_tiles = ty.n_tiles;
+  }
   const int q_tile0 = 2 * pair;
-  if (q_tile0 >= ty.n_tiles) return;  // whole CTA: this window type has fewer query tiles
-  const bool has_q1 = q_tile0 + 1 < ty.n_tiles;
+  if (q_tile0 >= n_q_tiles) return;  // whole CTA: this window type has fewer query tiles
+  const bool has_q1 = q_tile0 + 1 < n_q_tiles;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -340,6 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     }
     ptx::mbar_init(&c.drain, 1);
     c.abort = 0;
+    c.tile0 = P.dense ? split * P.split_tiles : 0;
+    c.ntile = P.dense ? min(P.split_tiles, (P.dense_rows + kTileRows - 1) / kTileRows - c.tile0) : 0;
     c.wtype[0] = wtype;
     c.org[0][0] = ot; c.org[0][1] = oy; c.org[0][2] = ox;
     for (int r = 0; r < P.routed_k; ++r) {
@@ -377,13 +397,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     if (lane == 0) {
       Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, true};
       Waiter drain{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
-      // a tile's TMA boxes deliver 256 bytes per valid row (two 128-byte halves)
-      uint32_t qbytes = uint32_t(P.plan.tile[ty.first_tile + q_tile0].valid_rows) * 256u;
-      if (has_q1) qbytes += uint32_t(P.plan.tile[ty.first_tile + q_tile0 + 1].valid_rows) * 256u;
-      ptx::mbar_arrive_expect_tx(&c.q_full, qbytes);
-      for (int g = 0; g < (has_q1 ? 2 : 1); ++g)
-        load_window_tile(P, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh, smem + kSmemQ + g * kTileBytes,
-                         &c.q_full);
+      if (P.dense) {
+        // whole 128-row boxes (rows past the end read as zero and still count)
+        ptx::mbar_arrive_expect_tx(&c.q_full, (has_q1 ? 2u : 1u) * kTileBytes);
+        for (int g = 0; g < (has_q1 ? 2 : 1); ++g) {
+          uint8_t *dst = smem + kSmemQ + g * kTileBytes;
+          ptx::tma_load_3d(dst, &P.map_qd, &c.q_full, 0, (q_tile0 + g) * kTileRows, bh);
+          ptx::tma_load_3d(dst + kHalfBytes, &P.map_qd, &c.q_full, 64, (q_tile0 + g) * kTileRows, bh);
+        }
+      } else {
+        // a tile's TMA boxes deliver 256 bytes per valid row (two 128-byte halves)
+        uint32_t qbytes = uint32_t(P.plan.tile[ty.first_tile + q_tile0].valid_rows) * 256u;
+        if (has_q1) qbytes += uint32_t(P.plan.tile[ty.first_tile + q_tile0 + 1].valid_rows) * 256u;
+        ptx::mbar_arrive_expect_tx(&c.q_full, qbytes);
+        for (int g = 0; g < (has_q1 ? 2 : 1); ++g)
+          load_window_tile(P, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh,
+                           smem + kSmemQ + g * kTileBytes, &c.q_full);
+      }
       KeyIter it = first_key(P, c);
       int last = -1;
       bool skipped0 = false;
@@ -590,7 +620,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       }
       ptx::fence_proxy_async_smem();
     }
-    if (ok && P.lse != nullptr) {
+    if (ok && P.lse != nullptr && P.dense) {
+      const int qrow = (q_tile0 + g) * kTileRows + row;
+      if (active && qrow < P.n_text)
+        P.lse[((long long)split * P.bh_count + bh) * P.n_text + qrow] = (m + log2f(l)) * 0.6931471805599453f;
+    } else if (ok && P.lse != nullptr) {
       // log-sum-exp of this row: m and l are in base 2 of the scaled scores
       const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
       for (int i = 0; i < tile.n_pieces; ++i) {
@@ -604,7 +638,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       }
     }
     ptx::named_barrier(1 + g, 128);
-    if (active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
+    if (P.dense && active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
+      // rows past n_text fall outside the output map and are not written
+      const int orow = (q_tile0 + g) * kTileRows, ob = split * P.bh_count + bh;
+      ptx::tma_store_3d(&P.map_od, q_tile, 0, orow, ob);
+      ptx::tma_store_3d(&P.map_od, q_tile + kHalfBytes, 64, orow, ob);
+      ptx::tma_store_commit();
+      ptx::tma_store_wait_read_all();
+    } else if (active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
       const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
       for (int i = 0; i < tile.n_pieces; ++i) {
         const PlanPiece pc = P.plan.piece[tile.first_piece + i];
@@ -656,6 +697,33 @@ bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, lon
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+basa_status run_attn(const AttnParams &P, long long blocks, cudaStream_t s) {
+  static const int emu = [] {
+    // tuning override for the share of exponentials done on the FMA pipe (pairs of 8)
+    const char *e = std::getenv("BASA_TUNE_EXP_EMU");
+    const int v = e ? std::atoi(e) : kDefaultEmuPairs;
+    return (v == 0 || v == 2) ? v : kDefaultEmuPairs;
+  }();
+  // Measured on B200 (FLUX 2048^2): every share of FMA-pipe exponentials tried (1/8 to 1/2)
+  // was slower than MUFU only, so 0 is the default; the variant stays for other parts/shapes.
+  auto kernel = emu == 2 ? attn_bf16_kernel<2> : attn_bf16_kernel<0>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    return BASA_ERR_CUDA;
+  kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+
+// Number of key-range splits for the text-query rows: enough CTAs to cover the SMs
+// once (one CTA per SM fits), at least 4 key tiles per split.
+int text_splits(const basa_params &p, int sms) {
+  const long long base = (long long)p.B * p.heads * (((p.n_text + kTileRows - 1) / kTileRows + 1) / 2);
+  const long long rows = (long long)p.T * p.H * p.W + p.n_text;
+  const int tiles = int((rows + kTileRows - 1) / kTileRows);
+  if (base >= sms) return 1;
+  return std::max(1, std::min<int>(int(sms / base), std::min(kMaxTextSplits, tiles / 4)));
+}
+
 }  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -669,6 +737,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+int device_sm_count() {
+  static int n[64] = {0};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n[dev] = 0;
+  return n[dev];
 }
 
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
@@ -702,6 +781,7 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
   P.n_text_tiles = (keys & BASA_KEYS_TEXT) ? (p.n_text + kTileRows - 1) / kTileRows : 0;
   P.use_windows = (keys & BASA_KEYS_WINDOWS) ? 1 : 0;
   P.lse = lse;
+  P.text_row0 = int(N);
   P.route = route_idx;
   P.dev_err = p.dev_err;
   P.routed_k = p.routed_k;
@@ -712,19 +792,68 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
   P.timeout_ns = (p.wait_timeout_us ? (unsigned long long)p.wait_timeout_us : 2000000ull) * 1000ull;
   const long long blocks = (long long)p.B * p.heads * P.g.nWin * P.plan.max_pairs;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
-  static const int emu = [] {
-    // tuning override for the share of exponentials done on the FMA pipe (pairs of 8)
-    const char *e = std::getenv("BASA_TUNE_EXP_EMU");
-    const int v = e ? std::atoi(e) : kDefaultEmuPairs;
-    return (v == 0 || v == 2) ? v : kDefaultEmuPairs;
-  }();
-  // Measured on B200 (FLUX 2048^2): every share of FMA-pipe exponentials tried (1/8 to 1/2)
-  // was slower than MUFU only, so 0 is the default; the variant stays for other parts/shapes.
-  auto kernel = emu == 2 ? attn_bf16_kernel<2> : attn_bf16_kernel<0>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  return run_attn(P, blocks, s);
+}
+
+size_t text_attn_workspace(const basa_params &p, int sms) {
+  const int splits = text_splits(p, sms);
+  if (splits <= 1) return 0;
+  const size_t rows = size_t(splits) * p.B * p.heads * p.n_text;
+  return rows * p.head_dim * 2 + rows * sizeof(float);  // partial outputs (bf16), then their log-sum-exp
+}
+
+basa_status launch_attn_text_bf16(const void *q_text, const void *k, const void *v, void *out_text, void *workspace,
+                                  const basa_params &p, int sms, cudaStream_t s) {
+  if (!encode_fn()) return BASA_ERR_CUDA;
+  AttnParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.g = make_geo(p);
+  const long long N = P.g.N;
+  const long long kv_rows = N + p.n_text;
+  const int bh = p.B * p.heads;
+  const int splits = text_splits(p, sms);
+  uint8_t *part = static_cast<uint8_t *>(workspace);
+  float *part_lse = reinterpret_cast<float *>(part + size_t(splits) * bh * p.n_text * p.head_dim * 2);
+  if (!encode_rows_map(&P.map_kt, k, p, kv_rows) || !encode_rows_map(&P.map_vt, v, p, kv_rows) ||
+      !encode_rows_map(&P.map_qd, q_text, p, p.n_text))
     return BASA_ERR_CUDA;
-  kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
-  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+  // outputs: straight to out_text, or per-split partials [split][b*head][n_text][d]
+  basa_params po = p;
+  po.B = 1;
+  po.heads = splits * bh;
+  if (!encode_rows_map(&P.map_od, splits > 1 ? static_cast<const void *>(part) : out_text, splits > 1 ? po : p,
+                       p.n_text))
+    return BASA_ERR_CUDA;
+  P.dense = 1;
+  P.dense_rows = int(kv_rows);
+  P.dense_q_tiles = (p.n_text + kTileRows - 1) / kTileRows;
+  P.dense_pairs = (P.dense_q_tiles + 1) / 2;
+  const int key_tiles = int((kv_rows + kTileRows - 1) / kTileRows);
+  P.n_splits = splits;
+  P.split_tiles = (key_tiles + splits - 1) / splits;
+  P.n_splits = (key_tiles + P.split_tiles - 1) / P.split_tiles;  // no empty split
+  P.bh_count = bh;
+  P.n_text = p.n_text;
+  P.routed_k = 0;
+  P.use_windows = 0;
+  P.text_row0 = 0;
+  P.lse = P.n_splits > 1 ? part_lse : nullptr;
+  P.dev_err = p.dev_err;
+  P.scale_log2 = float(1.4426950408889634 / std::sqrt(double(p.head_dim)));
+  P.flags = p.flags;
+  P.all_full = kv_rows % kTileRows == 0;
+  P.timeout_ns = (p.wait_timeout_us ? (unsigned long long)p.wait_timeout_us : 2000000ull) * 1000ull;
+  const long long blocks = (long long)bh * P.dense_pairs * P.n_splits;
+  if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
+  basa_status st = run_attn(P, blocks, s);
+  if (st != BASA_OK || P.n_splits == 1) return st;
+  const void *outs[kMaxTextSplits];
+  const float *lses[kMaxTextSplits];
+  for (int i = 0; i < P.n_splits; ++i) {
+    outs[i] = part + size_t(i) * bh * p.n_text * p.head_dim * 2;
+    lses[i] = part_lse + size_t(i) * bh * p.n_text;
+  }
+  return launch_merge_rows(P.n_splits, outs, lses, out_text, nullptr, (long long)bh * p.n_text, p.head_dim, p.dtype, s);
 }
 
 }  // namespace basa

@@ -21,6 +21,7 @@ struct F32Args {
   Geo g;
   int heads, d, n_text, n_pool, routed_k, win_tok, q_chunks;
   int n_vis_keys, n_pool_keys, n_text_keys;  // keys taken from each group (0 = group not selected)
+  int dense;  // text-query rows: queries are q_text rows, keys are all N + n_text rows of k, v
   float scale;
 };
 
@@ -30,6 +31,7 @@ __device__ __forceinline__ const float *key_row(const F32Args &a, const float *k
                                                 const int *wins, int j) {
   const int nvis = a.n_vis_keys;
   const long long rows = (long long)a.g.N + a.n_text;
+  if (a.dense) return kv + (bh * rows + j) * a.d;
   if (j < nvis) {
     const int u = wins[j / a.win_tok];
     const int l = j % a.win_tok;
@@ -53,33 +55,38 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(F32Args a) {
   __shared__ float vs[kKeyTile][D];
   __shared__ int wins[1 + kMaxRouted];
 
+  const int n_win = a.dense ? 1 : a.g.nWin;
   const int chunk = blockIdx.x % a.q_chunks;
-  const int w = (blockIdx.x / a.q_chunks) % a.g.nWin;
-  const long long bh = blockIdx.x / (a.q_chunks * a.g.nWin);
+  const int w = (blockIdx.x / a.q_chunks) % n_win;
+  const long long bh = blockIdx.x / (a.q_chunks * n_win);
   if (threadIdx.x == 0) wins[0] = w;
-  if (threadIdx.x > 0 && threadIdx.x <= a.routed_k)
+  if (!a.dense && threadIdx.x > 0 && threadIdx.x <= a.routed_k)
     wins[threadIdx.x] = a.route[(bh * a.g.nWin + w) * a.routed_k + threadIdx.x - 1];
   __syncthreads();
 
   const int half = threadIdx.x % TPQ;
   const int lq = chunk * QPB + threadIdx.x / TPQ;
-  const bool active = lq < a.win_tok;
-  int ot, oy, ox, type;
-  window_origin(a.g, w, &ot, &oy, &ox, &type);
+  const bool active = lq < (a.dense ? a.n_text : a.win_tok);
+  // query / output row inside this (b, head): a token of the grid, or a text row
+  const long long q_rows = a.dense ? a.n_text : a.g.N;
   long long qtok = 0;
-  if (active) {
+  if (active && a.dense) {
+    qtok = lq;
+  } else if (active) {
+    int ot, oy, ox, type;
+    window_origin(a.g, w, &ot, &oy, &ox, &type);
     const int lt = lq / (a.g.wh * a.g.ww), ly = (lq / a.g.ww) % a.g.wh, lx = lq % a.g.ww;
     qtok = ((long long)((ot + lt) % a.g.T) * a.g.H + (oy + ly) % a.g.H) * a.g.W + (ox + lx) % a.g.W;
   }
   float q[64], o[64];
-  const float *qp = a.q + (bh * a.g.N + qtok) * D;
+  const float *qp = a.q + (bh * q_rows + qtok) * D;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     q[i] = active ? qp[i * TPQ + half] * a.scale : 0.f;
     o[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int nk = a.n_vis_keys + a.n_pool_keys + a.n_text_keys;
+  const int nk = a.dense ? a.g.N + a.n_text : a.n_vis_keys + a.n_pool_keys + a.n_text_keys;
   for (int k0 = 0; k0 < nk; k0 += kKeyTile) {
     __syncthreads();
     for (int i = threadIdx.x; i < kKeyTile * (D / 4); i += kThreads) {
@@ -120,10 +127,10 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(F32Args a) {
   }
   if (active) {
     const float inv = 1.0f / l;
-    float *op = a.out + (bh * a.g.N + qtok) * D;
+    float *op = a.out + (bh * q_rows + qtok) * D;
 #pragma unroll
     for (int i = 0; i < 64; ++i) op[i * TPQ + half] = o[i] * inv;
-    if (a.lse && half == 0) a.lse[bh * a.g.N + qtok] = m + logf(l);
+    if (a.lse && half == 0) a.lse[bh * q_rows + qtok] = m + logf(l);
   }
 }
 
@@ -155,6 +162,28 @@ basa_status launch_attn_f32(const void *q, const void *k, const void *v, const v
   a.q_chunks = (a.win_tok + qpb - 1) / qpb;
   a.scale = 1.0f / sqrtf(float(p.head_dim));
   const long long blocks = (long long)p.B * p.heads * a.g.nWin * a.q_chunks;
+  if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
+  if (p.head_dim == 64) attn_f32_kernel<64><<<unsigned(blocks), kThreads, 0, s>>>(a);
+  else attn_f32_kernel<128><<<unsigned(blocks), kThreads, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+basa_status launch_attn_text_f32(const void *q_text, const void *k, const void *v, void *out_text,
+                                 const basa_params &p, cudaStream_t s) {
+  F32Args a{};
+  a.q = static_cast<const float *>(q_text);
+  a.k = static_cast<const float *>(k);
+  a.v = static_cast<const float *>(v);
+  a.out = static_cast<float *>(out_text);
+  a.g = make_geo(p);
+  a.heads = p.heads;
+  a.d = p.head_dim;
+  a.n_text = p.n_text;
+  a.dense = 1;
+  const int qpb = kThreads / (p.head_dim / 64);
+  a.q_chunks = (p.n_text + qpb - 1) / qpb;
+  a.scale = 1.0f / sqrtf(float(p.head_dim));
+  const long long blocks = (long long)p.B * p.heads * a.q_chunks;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
   if (p.head_dim == 64) attn_f32_kernel<64><<<unsigned(blocks), kThreads, 0, s>>>(a);
   else attn_f32_kernel<128><<<unsigned(blocks), kThreads, 0, s>>>(a);

@@ -143,5 +143,16 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
 // out = sum_b exp(lse_b - L) out_b, L = log sum_b exp(lse_b), over n branches.
 basa_status launch_merge(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
                          const basa_params &p, cudaStream_t s);
+// The same over `rows` rows of head_dim elements, n <= kMaxMerge.
+constexpr int kMaxMerge = 8;
+basa_status launch_merge_rows(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
+                              long long rows, int head_dim, basa_dtype dtype, cudaStream_t s);
+// Text-query rows (dense attention of the n_text text queries over all k/v rows).
+int device_sm_count();
+size_t text_attn_workspace(const basa_params &p, int sms);  // bf16 path; 0 = none needed
+basa_status launch_attn_text_bf16(const void *q_text, const void *k, const void *v, void *out_text, void *workspace,
+                                  const basa_params &p, int sms, cudaStream_t s);
+basa_status launch_attn_text_f32(const void *q_text, const void *k, const void *v, void *out_text,
+                                 const basa_params &p, cudaStream_t s);
 
 }  // namespace basa

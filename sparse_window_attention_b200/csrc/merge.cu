@@ -10,8 +10,8 @@ namespace basa {
 namespace {
 
 struct MergeArgs {
-  const void *out[BASA_MAX_BRANCHES];
-  const float *lse[BASA_MAX_BRANCHES];
+  const void *out[kMaxMerge];
+  const float *lse[kMaxMerge];
   int n;
   void *dst;
   float *dst_lse;
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
   const long long row = idx / a.lpr;
   const int c = int(idx % a.lpr);
   if (row >= a.rows) return;
-  float L[BASA_MAX_BRANCHES];
+  float L[kMaxMerge];
   float m = -INFINITY;
   for (int b = 0; b < a.n; ++b) {
     L[b] = a.lse[b][row];
@@ -77,8 +77,9 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
 
 }  // namespace
 
-basa_status launch_merge(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
-                         const basa_params &p, cudaStream_t s) {
+basa_status launch_merge_rows(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
+                              long long rows, int head_dim, basa_dtype dtype, cudaStream_t s) {
+  if (n < 1 || n > kMaxMerge) return BASA_ERR_INVALID_ARG;
   MergeArgs a{};
   for (int b = 0; b < n; ++b) {
     a.out[b] = outs[b];
@@ -87,15 +88,20 @@ basa_status launch_merge(int n, const void *const *outs, const float *const *lse
   a.n = n;
   a.dst = out;
   a.dst_lse = lse;
-  a.rows = (long long)p.B * p.heads * p.T * p.H * p.W;
-  a.d = p.head_dim;
-  a.lpr = p.head_dim * (p.dtype == BASA_BF16 ? 2 : 4) / 16;
+  a.rows = rows;
+  a.d = head_dim;
+  a.lpr = head_dim * (dtype == BASA_BF16 ? 2 : 4) / 16;
   const long long threads = a.rows * a.lpr;
   const long long blocks = (threads + 255) / 256;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
-  if (p.dtype == BASA_BF16) merge_kernel<__nv_bfloat16><<<unsigned(blocks), 256, 0, s>>>(a);
+  if (dtype == BASA_BF16) merge_kernel<__nv_bfloat16><<<unsigned(blocks), 256, 0, s>>>(a);
   else merge_kernel<float><<<unsigned(blocks), 256, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
+}
+
+basa_status launch_merge(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
+                         const basa_params &p, cudaStream_t s) {
+  return launch_merge_rows(n, outs, lses, out, lse, (long long)p.B * p.heads * p.T * p.H * p.W, p.head_dim, p.dtype, s);
 }
 
 }  // namespace basa

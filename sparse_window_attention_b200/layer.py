@@ -107,6 +107,16 @@ class BasaLayer:
         self.merge([o for o, _ in bufs], [l for _, l in bufs], out, None, stream)
         return out
 
+    def text_attention(self, q_text, k, v, out_text, stream=None):
+        """Output rows of the text queries (dense over all keys; basa_text_attn_fwd)."""
+        nbytes = B.basa_text_attn_workspace_bytes(self.params((0, 0, 0)))
+        ws = None
+        if nbytes > 0:
+            if getattr(self, "text_workspace", None) is None or self.text_workspace.numel() < nbytes:
+                self.text_workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            ws = self.text_workspace
+        B.basa_text_attn_fwd(q_text, k, v, out_text, ws, self.params((0, 0, 0)), stream)
+
     def forward(self, q, k, v, shift, out=None, stream=None):
         """Full layer: pooled K/V, routed windows (if routed_k > 0), attention."""
         if out is None:

@@ -160,6 +160,15 @@ def test_branch_form_checks():
     assert merge([FAKE], [FAKE], out=None) == 1
 
 
+def test_text_attn_checks():
+    p = _p()
+    assert B.basa_text_attn_fwd(FAKE, FAKE, FAKE, FAKE, None, _p(n_text=0), stream=0, check=False) == 1
+    assert B.basa_text_attn_fwd(FAKE + 8, FAKE, FAKE, FAKE, None, p, stream=0, check=False) == 1
+    assert B.basa_text_attn_fwd(FAKE, FAKE, FAKE, None, None, p, stream=0, check=False) == 1
+    assert B.basa_text_attn_fwd(FAKE, FAKE, FAKE, FAKE, None, _p(head_dim=64), stream=0, check=False) == 3
+    assert B.basa_text_attn_workspace_bytes(_p(n_text=0)) == 0
+
+
 def test_route_workspace_bytes():
     p = _p(routed_k=2)
     assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4
