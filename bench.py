@@ -263,10 +263,38 @@ def run_ours(args, world, rank, local):
         res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world)
     if not args.no_extra and world == 1:
         res["branch_form"] = run_branch_form(args, layer, qd, kd, vd, shifts, flops)
+        if wl.n_text > 0:
+            res["text_queries"] = run_text_queries(args, layer, wl, kd, vd)
         for name in ("wan", "wan_video"):
             if args.workload != name:
                 res["also_" + name] = run_also(args, name)
     return res
+
+
+def run_text_queries(args, layer, wl, kd, vd):
+    """The text-query rows of the joint layer: dense attention of the n_text text
+    queries over all N + n_text keys (4 d FLOPs per query-key pair)."""
+    g = torch.Generator(device="cpu").manual_seed(args.seed + 100)
+    qt = torch.randn(wl.B, wl.heads, wl.n_text, wl.d, generator=g).to(kd.dtype).cuda()
+    out = torch.empty_like(qt)
+    steps = max(20, args.steps // 4)
+    for _ in range(3):
+        layer.text_attention(qt, kd, vd, out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        layer.text_attention(qt, kd, vd, out)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    flops = 4.0 * wl.d * wl.B * wl.heads * wl.n_text * (wl.N + wl.n_text)
+    peaks, _ = load_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"ms": round(ms, 4), "gflop": round(flops / 1e9, 2), "value": round(achieved, 2), "unit": "TFLOP/s",
+            "frac_of_measured_bf16": round(achieved / peaks["bf16_tflops"], 4),
+            "workspace_bytes": layer.text_workspace.numel() if getattr(layer, "text_workspace", None) is not None else 0}
 
 
 def run_branch_form(args, layer, qd, kd, vd, shifts, flops):
