@@ -367,6 +367,97 @@ def text_query_attention(q_text, k, v, geo: Geometry):
     return out
 
 
+def basa_attention_backward(q, k, v, geo: Geometry, dout, route_idx=None):
+    """Gradients of the BASA forward w.r.t. q, k and v for an output gradient dout.
+
+    Differentiates basa_attention step by step (routing is a selection and is held
+    fixed at route_idx; the pooled K/V are means of k, v and pass their gradient
+    back to every token of the patch). Per query block of window w, with keys
+    Kc = [own | routed | pooled | text] and P = softmax(Q Kc^T / sqrt(d)):
+      dVc = P^T dO,  dP = dO Vc^T,  dS = P * (dP - rowsum(dP * P)),
+      dQ = dS Kc / sqrt(d),  dKc = dS^T Q / sqrt(d);
+    the rows of dKc, dVc are then added back to the tokens they came from.
+    Returns (dq [B,h,N,d], dk, dv [B,h,N+n_text,d]) float64.
+    """
+    q64 = np.asarray(q, dtype=np.float64)
+    k64 = np.asarray(k, dtype=np.float64)
+    v64 = np.asarray(v, dtype=np.float64)
+    do64 = np.asarray(dout, dtype=np.float64)
+    B, h, N, d = q64.shape
+    if geo.routed_k > 0 and route_idx is None:
+        route_idx, _ = route_windows(q64, k64, geo)
+    kp = vp = None
+    if geo.has_pool:
+        kp, vp = pool_kv(k64, v64, geo)
+
+    def windows(x):
+        return window_partition(cyclic_shift(to_grid(x[:, :, :N], geo.grid), geo.shift), geo.window)
+
+    Qw, Kw, Vw, dOw = windows(q64), windows(k64), windows(v64), windows(do64)
+    dQw = np.zeros_like(Qw)
+    dKw = np.zeros_like(Kw)
+    dVw = np.zeros_like(Vw)
+    dkp = np.zeros((B, h, geo.n_pool, d))
+    dvp = np.zeros((B, h, geo.n_pool, d))
+    dk_text = np.zeros((B, h, geo.n_text, d))
+    dv_text = np.zeros((B, h, geo.n_text, d))
+    scale = 1.0 / np.sqrt(d)
+    wt = geo.win_tokens
+    for b in range(B):
+        for hh in range(h):
+            for w in range(geo.n_win):
+                wins = [w] + [int(route_idx[b, hh, w, r]) for r in range(geo.routed_k)]
+                kparts = [Kw[b, hh, u] for u in wins]
+                vparts = [Vw[b, hh, u] for u in wins]
+                if geo.has_pool:
+                    kparts.append(kp[b, hh])
+                    vparts.append(vp[b, hh])
+                if geo.n_text > 0:
+                    kparts.append(k64[b, hh, N:])
+                    vparts.append(v64[b, hh, N:])
+                Kc = np.concatenate(kparts, axis=0)
+                Vc = np.concatenate(vparts, axis=0)
+                Qb, dOb = Qw[b, hh, w], dOw[b, hh, w]
+                s = (Qb @ Kc.T) * scale
+                s = s - s.max(axis=1, keepdims=True)
+                P = np.exp(s)
+                P = P / P.sum(axis=1, keepdims=True)
+                dVc = P.T @ dOb
+                dP = dOb @ Vc.T
+                dS = P * (dP - (dP * P).sum(axis=1, keepdims=True))
+                dQw[b, hh, w] = (dS @ Kc) * scale
+                dKc = (dS.T @ Qb) * scale
+                for i, u in enumerate(wins):
+                    dKw[b, hh, u] += dKc[i * wt:(i + 1) * wt]
+                    dVw[b, hh, u] += dVc[i * wt:(i + 1) * wt]
+                off = len(wins) * wt
+                if geo.has_pool:
+                    dkp[b, hh] += dKc[off:off + geo.n_pool]
+                    dvp[b, hh] += dVc[off:off + geo.n_pool]
+                    off += geo.n_pool
+                if geo.n_text > 0:
+                    dk_text[b, hh] += dKc[off:]
+                    dv_text[b, hh] += dVc[off:]
+
+    def unwindows(xw):
+        X = inverse_cyclic_shift(window_unpartition(xw, geo.grid, geo.window), geo.shift)
+        return X.reshape(B, h, N, d)
+
+    dq = unwindows(dQw)
+    dk_vis, dv_vis = unwindows(dKw), unwindows(dVw)
+    if geo.has_pool:
+        # kp = mean over the patch: each token of patch P receives dkp[P] / |P|
+        T, H, W = geo.grid
+        pt, ph, pw = geo.pool
+        for g_vis, g_pool in ((dk_vis, dkp), (dv_vis, dvp)):
+            G = g_pool.reshape(B, h, T // pt, H // ph, W // pw, d) / (pt * ph * pw)
+            G = np.repeat(np.repeat(np.repeat(G, pt, axis=2), ph, axis=3), pw, axis=4)
+            g_vis += G.reshape(B, h, N, d)
+    dk = np.concatenate([dk_vis, dk_text], axis=2)
+    dv = np.concatenate([dv_vis, dv_text], axis=2)
+    return dq, dk, dv
+
+
 def window_of_token(geo: Geometry):
     """Window id of every token of the ORIGINAL grid, computed without any roll.
 

@@ -499,3 +499,52 @@ def test_text_queries_zero_query_is_mean_of_all_values():
     v = rng.standard_normal((1, 2, geo.N + 3, 8))
     out = O.text_query_attention(np.zeros((1, 2, 3, 8)), k, v, geo)
     np.testing.assert_allclose(out, np.broadcast_to(v.mean(axis=2, keepdims=True), out.shape), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+
+
+BWD_GEOS = [
+    O.Geometry(grid=(1, 8, 8), window=(1, 4, 4), shift=(0, 2, 2), pool=(1, 2, 2), n_text=3, routed_k=2),
+    O.Geometry(grid=(4, 4, 6), window=(2, 2, 3), shift=(1, 1, 2), pool=(2, 2, 3), routed_k=1),
+]
+
+
+@pytest.mark.parametrize("geo", BWD_GEOS)
+def test_backward_matches_finite_differences(geo):
+    """Central differences of L = sum(dout * out) w.r.t. sampled entries of q, k, v
+    (routing held fixed, pooling recomputed from k and v)."""
+    q, k, v = _qkv(geo, B=1, h=1, d=4, seed=41)
+    rng = np.random.default_rng(3)
+    dout = rng.standard_normal(q.shape)
+    route = O.route_windows(q, k, geo)[0] if geo.routed_k else None
+    dq, dk, dv = O.basa_attention_backward(q, k, v, geo, dout, route_idx=route)
+
+    def loss(qq, kk, vv):
+        return float((dout * O.basa_attention(qq, kk, vv, geo, route_idx=route)).sum())
+
+    eps = 1e-5
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in [tuple(rng.integers(0, s) for s in x.shape) for _ in range(12)]:
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            lp = loss(*[xp if a is x else a for a in args])
+            lm = loss(*[xm if a is x else a for a in args])
+            num = (lp - lm) / (2 * eps)
+            assert abs(num - g[idx]) <= 1e-7 + 1e-6 * abs(num), (name, idx, num, g[idx])
+
+
+def test_backward_whole_grid_is_sdpa_autograd():
+    """window = grid, shift 0, with text keys: float64 autograd through torch SDPA."""
+    geo = O.Geometry(grid=(2, 4, 6), window=(2, 4, 6), n_text=4)
+    q, k, v = _qkv(geo, B=1, h=2, d=8, seed=43)
+    dout = np.random.default_rng(9).standard_normal(q.shape)
+    dq, dk, dv = O.basa_attention_backward(q, k, v, geo, dout)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)
+    out.backward(torch.from_numpy(dout))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-12)

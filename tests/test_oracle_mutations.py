@@ -37,6 +37,9 @@ MUTATIONS = [
     ("branch drops routed", "for u in [w] + [int(route_idx[b, hh, w, r]) for r in range(geo.routed_k)]:", "for u in [w]:", ["branch_merge", "lse_zero_q"]),
     ("text queries skip text keys", "            s = (qt[b, hh] @ k64[b, hh].T) / np.sqrt(d)", "            s = (qt[b, hh] @ k64[b, hh, : geo.N].T) / np.sqrt(d)", ["text_sdpa", "text_zero_q"]),
     ("text queries scale", "            s = (qt[b, hh] @ k64[b, hh].T) / np.sqrt(d)", "            s = (qt[b, hh] @ k64[b, hh].T) / d", ["text_sdpa"]),
+    ("bwd softmax term", "dS = P * (dP - (dP * P).sum(axis=1, keepdims=True))", "dS = P * dP", ["bwd_fd", "bwd_sdpa"]),
+    ("bwd pool spread", "G = g_pool.reshape(B, h, T // pt, H // ph, W // pw, d) / (pt * ph * pw)", "G = g_pool.reshape(B, h, T // pt, H // ph, W // pw, d)", ["bwd_fd"]),
+    ("bwd routed keys", "                    dKw[b, hh, u] += dKc[i * wt:(i + 1) * wt]", "                    dKw[b, hh, w] += dKc[i * wt:(i + 1) * wt]", ["bwd_fd"]),
     ("unshift output", "O = inverse_cyclic_shift(window_unpartition(Ow, geo.grid, geo.window), geo.shift)", "O = window_unpartition(Ow, geo.grid, geo.window)", ["dense_masked"]),
 ]
 
@@ -58,6 +61,8 @@ PINS = {
     "rows_sum": lambda: [pins.test_softmax_rows_sum_to_one(g) for g in pins.TINY_GEOS],
     "lse_scipy": lambda: pins.test_lse_whole_grid_is_scipy_logsumexp(),
     "text_sdpa": lambda: pins.test_text_queries_dense_sdpa(),
+    "bwd_fd": lambda: [pins.test_backward_matches_finite_differences(g) for g in pins.BWD_GEOS],
+    "bwd_sdpa": lambda: pins.test_backward_whole_grid_is_sdpa_autograd(),
     "text_zero_q": lambda: pins.test_text_queries_zero_query_is_mean_of_all_values(),
     "lse_zero_q": lambda: pins.test_lse_of_zero_queries_is_log_of_key_count(),
     "branch_merge": lambda: [pins.test_branches_merge_to_the_joint_softmax(g) for g in pins.TINY_GEOS],
