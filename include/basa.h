@@ -228,6 +228,31 @@ basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v,
                                basa_stream_t stream);
 
 /*
+ * basa_window_attn_bwd — gradients of basa_window_attn_fwd with respect to q, k
+ * and v, for the training step of the dense-teacher adaptation (BASA §3.4).
+ *
+ * Inputs: the forward's arguments, its output `out` and the log-sum-exp `lse`
+ * of basa_window_attn_fwd_lse with BASA_KEYS_ALL, and the output gradient
+ * `dout` [B, heads, N, head_dim]. With P = softmax(q K^T / sqrt(d)) over each
+ * query's keys and D_i = dout_i . out_i:
+ *   dS = P (dout V^T - D),  dq = dS K / sqrt(d),  dK = dS^T q / sqrt(d),  dV = P^T dout,
+ * the key rows of dK, dV added back to the tokens they came from: own and routed
+ * window tokens, text rows, and pooled keys spread evenly over their patch's
+ * tokens (kp, vp are means). Routing is a selection and passes no gradient.
+ * Outputs (overwritten): dq [B, heads, N, d], dk, dv [B, heads, N + n_text, d].
+ * Float32 only, head_dim 128 (BASA_ERR_UNSUPPORTED otherwise). `workspace`
+ * (device, 16-byte aligned) holds basa_window_attn_bwd_workspace_bytes(p) bytes
+ * for the pooled keys' gradients (NULL when that is 0). dk, dv are accumulated
+ * with atomic adds, so their last bits can differ between runs; dq cannot.
+ */
+size_t basa_window_attn_bwd_workspace_bytes(const basa_params *p);
+basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v,
+                                 const void *kp, const void *vp, const int32_t *route_idx,
+                                 const void *out, const float *lse, const void *dout,
+                                 void *dq, void *dk, void *dv, void *workspace,
+                                 const basa_params *p, basa_stream_t stream);
+
+/*
  * basa_merge_branches — joint softmax from n branch results (BASA §A.1).
  *
  *   L[r]   = log sum_b exp(lses[b][r])

@@ -39,6 +39,8 @@ EXPORTED = (
     "basa_merge_branches",
     "basa_text_attn_workspace_bytes",
     "basa_text_attn_fwd",
+    "basa_window_attn_bwd_workspace_bytes",
+    "basa_window_attn_bwd",
     "basa_status_string",
     "basa_device_error_status",
 )
@@ -94,6 +96,10 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.basa_text_attn_workspace_bytes.restype = ctypes.c_size_t
     lib.basa_text_attn_fwd.argtypes = [vp, vp, vp, vp, vp, P, vp]
     lib.basa_text_attn_fwd.restype = ctypes.c_int
+    lib.basa_window_attn_bwd_workspace_bytes.argtypes = [P]
+    lib.basa_window_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.basa_window_attn_bwd.argtypes = [vp] * 13 + [P, vp]
+    lib.basa_window_attn_bwd.restype = ctypes.c_int
     lib.basa_status_string.argtypes = [ctypes.c_int]
     lib.basa_status_string.restype = ctypes.c_char_p
     lib.basa_device_error_status.argtypes = [ctypes.c_int32]
@@ -228,4 +234,17 @@ def basa_text_attn_fwd(q_text, k, v, out_text, workspace, params: basa_params, s
                                  ctypes.byref(params), _stream(stream))
     if check:
         _check(st, "basa_text_attn_fwd")
+    return st
+
+
+def basa_window_attn_bwd_workspace_bytes(params: basa_params) -> int:
+    return _lib.basa_window_attn_bwd_workspace_bytes(ctypes.byref(params))
+
+
+def basa_window_attn_bwd(q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv, workspace, params: basa_params,
+                         stream=None, check=True) -> int:
+    st = _lib.basa_window_attn_bwd(*[_ptr(x) for x in (q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv,
+                                                        workspace)], ctypes.byref(params), _stream(stream))
+    if check:
+        _check(st, "basa_window_attn_bwd")
     return st

@@ -204,6 +204,32 @@ basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v,
   return basa::launch_attn_text_bf16(q_text, k, v, out_text, workspace, *p, sms, s);
 }
 
+size_t basa_window_attn_bwd_workspace_bytes(const basa_params *p) {
+  if (check_common(p) != BASA_OK) return 0;
+  return basa::attn_bwd_workspace(*p);
+}
+
+basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                                 const int32_t *route_idx, const void *out, const float *lse, const void *dout,
+                                 void *dq, void *dk, void *dv, void *workspace, const basa_params *p,
+                                 basa_stream_t stream) {
+  basa_status st = check_common(p);
+  if (st != BASA_OK) return st;
+  if (p->dtype != BASA_F32 || p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (empty_batch(p)) return BASA_OK;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return BASA_ERR_INVALID_ARG;
+  if (has_pool(p) != (kp != nullptr) || has_pool(p) != (vp != nullptr)) return BASA_ERR_INVALID_ARG;
+  if ((p->routed_k > 0) != (route_idx != nullptr)) return BASA_ERR_INVALID_ARG;
+  for (const void *x : {q, k, v, out, dout, static_cast<const void *>(dq), static_cast<const void *>(dk),
+                        static_cast<const void *>(dv)})
+    if (!aligned16(x)) return BASA_ERR_INVALID_ARG;
+  if (!aligned4(lse) || (route_idx && !aligned4(route_idx))) return BASA_ERR_INVALID_ARG;
+  if (kp && (!aligned16(kp) || !aligned16(vp))) return BASA_ERR_INVALID_ARG;
+  if (basa::attn_bwd_workspace(*p) > 0 && (!workspace || !aligned16(workspace))) return BASA_ERR_INVALID_ARG;
+  return basa::launch_attn_bwd_f32(q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv, workspace, *p,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
 basa_status basa_merge_branches(int n, const void *const *outs, const float *const *lses, void *out, float *lse,
                                 const basa_params *p, basa_stream_t stream) {
   basa_status st = check_common(p);

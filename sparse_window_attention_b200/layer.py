@@ -117,6 +117,18 @@ class BasaLayer:
             ws = self.text_workspace
         B.basa_text_attn_fwd(q_text, k, v, out_text, ws, self.params((0, 0, 0)), stream)
 
+    def backward(self, q, k, v, out, lse, dout, shift, stream=None):
+        """dq, dk, dv of the attention (float32; basa_window_attn_bwd) for the pooled
+        K/V and routed windows currently held by the layer."""
+        dq = torch.empty_like(q)
+        dk = torch.empty_like(k)
+        dv = torch.empty_like(v)
+        nbytes = B.basa_window_attn_bwd_workspace_bytes(self.params(shift))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device) if nbytes else None
+        B.basa_window_attn_bwd(q, k, v, self.kp, self.vp, self.route_idx, out, lse, dout, dq, dk, dv, ws,
+                               self.params(shift), stream)
+        return dq, dk, dv
+
     def forward(self, q, k, v, shift, out=None, stream=None):
         """Full layer: pooled K/V, routed windows (if routed_k > 0), attention."""
         if out is None:

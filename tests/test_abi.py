@@ -169,6 +169,21 @@ def test_text_attn_checks():
     assert B.basa_text_attn_workspace_bytes(_p(n_text=0)) == 0
 
 
+def test_backward_checks():
+    pf = _p(dtype="f32")
+    args = [FAKE] * 5 + [None] + [FAKE] * 7
+    assert B.basa_window_attn_bwd(*args, _p(), stream=0, check=False) == 3  # bfloat16: not built
+    assert B.basa_window_attn_bwd(*args, _p(dtype="f32", head_dim=64), stream=0, check=False) == 3
+    bad = list(args)
+    bad[8] = None  # no dout
+    assert B.basa_window_attn_bwd(*bad, pf, stream=0, check=False) == 1
+    bad = list(args)
+    bad[9] = FAKE + 4  # misaligned dq
+    assert B.basa_window_attn_bwd(*bad, pf, stream=0, check=False) == 1
+    # pooled gradients: 2 x heads x 64 patches x 128 floats
+    assert B.basa_window_attn_bwd_workspace_bytes(pf) == 2 * 2 * 64 * 128 * 4
+
+
 def test_route_workspace_bytes():
     p = _p(routed_k=2)
     assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4
