@@ -265,6 +265,7 @@ def run_ours(args, world, rank, local):
         res["branch_form"] = run_branch_form(args, layer, qd, kd, vd, shifts, flops)
         if wl.n_text > 0:
             res["text_queries"] = run_text_queries(args, layer, wl, kd, vd)
+        res["backward_f32"] = run_backward(args)
         for name in ("wan", "wan_video"):
             if args.workload != name:
                 res["also_" + name] = run_also(args, name)
@@ -295,6 +296,43 @@ def run_text_queries(args, layer, wl, kd, vd):
     return {"ms": round(ms, 4), "gflop": round(flops / 1e9, 2), "value": round(achieved, 2), "unit": "TFLOP/s",
             "frac_of_measured_bf16": round(achieved / peaks["bf16_tflops"], 4),
             "workspace_bytes": layer.text_workspace.numel() if getattr(layer, "text_workspace", None) is not None else 0}
+
+
+def run_backward(args):
+    """Context: the float32 backward (CUDA cores) on the FLUX 1024^2 shape in float32,
+    counted as 10 d FLOPs per query-key pair (S recomputed, dP, dQ, dK, dV)."""
+    import dataclasses
+
+    from sparse_window_attention_b200 import binding as B
+    from sparse_window_attention_b200.layer import BasaLayer
+
+    wl = dataclasses.replace(synth.WORKLOADS["flux1k"], dtype="f32", name="flux1k_f32")
+    sh = (0, 8, 8)
+    q, k, v = synth.make_inputs(wl, seed=args.seed)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+    layer.pool_kv(kd, vd, sh)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=qd.device)
+    layer.attention_lse(qd, kd, vd, out, lse, sh, B.BASA_KEYS_ALL)
+    dout = torch.randn_like(qd)
+    for _ in range(2):
+        layer.backward(qd, kd, vd, out, lse, dout, sh)
+    torch.cuda.synchronize()
+    steps = 5
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        layer.backward(qd, kd, vd, out, lse, dout, sh)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    cnt = accounting.workload_counts(wl)
+    flops = 2.5 * cnt["attn_flops"]
+    return {"workload": "flux1k shape, float32, shift (0, 8, 8)", "ms": round(ms, 3),
+            "gflop": round(flops / 1e9, 2), "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "note": "CUDA-core float32 with atomic dK/dV accumulation; no tensor-core backward yet"}
 
 
 def run_branch_form(args, layer, qd, kd, vd, shifts, flops):
