@@ -301,13 +301,22 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_f32_kernel(BwdArgs b) {
       dpp += __shfl_xor_sync(0xffffffffu, dpp, 2);
       const float p = active ? expf(sp * a.scale - L) : 0.f;
       const float ds = p * (dpp - Drow);
+      // the 8 queries of a warp add to the same key row: sum them with shuffles
+      // (lanes l, l ^ 4, l ^ 8, l ^ 16 share a column) and let 4 lanes add to shared memory
+      const float dsq = active ? ds * a.scale : 0.f, pa = active ? p : 0.f;
 #pragma unroll
       for (int i = 0; i < C; ++i) {
         const int col = i * kBwdTPQ + part;
         dq[i] = fmaf(ds, ks[j][col], dq[i]);
-        if (active) {
-          atomicAdd(&dks[j][col], ds * a.scale * q[i]);
-          atomicAdd(&dvs[j][col], p * dout[i]);
+        float gk = dsq * q[i], gv = pa * dout[i];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          gk += __shfl_xor_sync(0xffffffffu, gk, off);
+          gv += __shfl_xor_sync(0xffffffffu, gv, off);
+        }
+        if ((threadIdx.x & 31) < kBwdTPQ) {
+          atomicAdd(&dks[j][col], gk);
+          atomicAdd(&dvs[j][col], gv);
         }
       }
     }

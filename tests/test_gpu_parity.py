@@ -279,6 +279,8 @@ SMALL = [
       route_radius=1),
     # radius two on a 6x6 window grid, float32
     W("f32_radius2", "f32", 1, 2, 64, (1, 24, 24), (1, 4, 4), (0, 2, 1), (1, 4, 4), 0, 8, "iid", route_radius=2),
+    # 1152 windows per head: staging of the candidates' means in several chunks
+    W("many_windows", "bf16", 1, 1, 128, (1, 128, 144), (1, 4, 4), (0, 2, 2), (0, 0, 0), 0, 2, "block_mean"),
 ]
 
 
