@@ -31,7 +31,8 @@ constexpr int kCellThreads = 256;
 constexpr int kMaxAxisRuns = 32;   // windows met by a box along one axis
 constexpr int kMaxAxisCells = 64;  // cells along one axis
 constexpr int kMaxCells = 96;      // cells of a box
-constexpr int kBoxTokens = 256;    // preferred box size
+constexpr int kBoxTokens = 512;    // preferred box size (tokens)
+constexpr size_t kSmemTwoCtas = 110 * 1024;  // shared memory that still fits two CTAs per SM
 
 // The windows one box meets along one axis: window index j and its (at most
 // two) runs of box-local coordinates [lo, hi). Two runs only when the box spans
@@ -405,9 +406,16 @@ static void axis_counts(int G, int e, int p, int w, int s, int *max_cells, int *
   }
 }
 
+static size_t cell_smem_bytes(int cells, int head_dim, basa_dtype dtype) {
+  const int vec = dtype == BASA_BF16 ? 8 : 4;
+  return ((sizeof(CellCtrl) + 15) & ~size_t(15)) + size_t(3) * vec * kCellThreads * sizeof(float) +
+         size_t(cells) * 3 * head_dim * sizeof(float);
+}
+
 // Box choice: whole pool patches per axis, extents dividing the grid; the x extent
-// is grown first (long contiguous rows), then y, then t, up to kBoxTokens tokens
-// (smaller while some box would have more than kMaxCells cells).
+// is grown first (long contiguous rows), then y, then t, up to kBoxTokens tokens,
+// halving the limit while some box would have more than kMaxCells cells or the
+// cell sums would keep two CTAs from sharing an SM (one pool patch is the floor).
 basa_status plan_fused(const basa_params &p, FusedPlan *fp) {
   const int G[3] = {p.T, p.H, p.W}, P[3] = {p.pt, p.ph, p.pw}, w[3] = {p.wt, p.wh, p.ww}, sh[3] = {p.st, p.sy, p.sx};
   for (int cap = kBoxTokens;; cap /= 2) {
@@ -435,6 +443,8 @@ basa_status plan_fused(const basa_params &p, FusedPlan *fp) {
       cells *= ca;
     }
     fits = fits && cells <= kMaxCells;
+    const bool single_patch = e[0] == P[0] && e[1] == P[1] && e[2] == P[2];
+    if (fits && !single_patch && cell_smem_bytes(int(cells), p.head_dim, p.dtype) > kSmemTwoCtas) fits = false;
     if (fits) {
       for (int ax = 0; ax < 3; ++ax) {
         fp->e[ax] = e[ax];
@@ -489,9 +499,7 @@ basa_status launch_pool_route_fused(const void *q, const void *k, const void *v,
   if (N * p.head_dim * esz >= (1ll << 32)) return BASA_ERR_UNSUPPORTED;  // 32-bit offsets inside a (b, head) slice
   const long long n_boxes = (long long)a.bh * fp.nb[0] * fp.nb[1] * fp.nb[2];
   if (n_boxes >= (1ll << 31) || 2ll * a.bh * g.nWin >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
-  const int vec = 16 / esz;
-  const size_t smem = ((sizeof(CellCtrl) + 15) & ~size_t(15)) + size_t(3) * vec * kCellThreads * sizeof(float) +
-                      size_t(fp.max_cells) * 3 * p.head_dim * sizeof(float);
+  const size_t smem = cell_smem_bytes(fp.max_cells, p.head_dim, p.dtype);
   auto kernel = p.dtype == BASA_BF16 ? cell_sum_kernel<__nv_bfloat16> : cell_sum_kernel<float>;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
