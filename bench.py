@@ -9,6 +9,15 @@ Rank 0 prints ONE JSON line. Multi-GPU runs (torchrun) give every rank its own
 copy of the workload (the path shards over (batch, head) with no exchange),
 time on the device and report the max over ranks ("scaling": "weak").
 
+The line also carries: `roofline` (the attention kernel's achieved TFLOP/s from
+CUDA events around its launches, against the measured bf16 peak, and its DRAM
+traffic from the committed ncu summary when that was taken on the current
+source), `hbm_kernels` (the pooling / routing pre-pass against measured HBM
+bandwidth), `e2e` (the same metric through BasaLayer.forward with pinned host
+buffers, copies of successive steps pipelined over three streams), `clocks`,
+`cpu_baseline` and context lines for the other workloads and forms (Wan 480p and
+video, the branch form, the text-query rows, the float32 backward).
+
 The reference arm (--impl reference) times the float64 CPU oracle on the host
 cores on a bounded sample of the same workload (the oracle is the only other
 implementation there is).

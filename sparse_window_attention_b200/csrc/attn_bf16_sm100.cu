@@ -19,6 +19,12 @@
 //               same (unshifted) coordinates the queries were loaded from.
 // Every wait is bounded (globaltimer); on expiry the kernel records a bit in
 // dev_err, drains its own in-flight copies and MMAs, frees TMEM and returns.
+//
+// The same kernel also serves the branch form (BASA §A.1): a key-group mask drops
+// the window, pooled or text segments from the key stream, and an optional
+// epilogue writes each query row's log-sum-exp; and the text-query rows, where the
+// queries are 128-row boxes of the text rows and the key stream is every k/v row,
+// split over CTA groups whose partial results are merged by log-sum-exp.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
