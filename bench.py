@@ -218,6 +218,11 @@ def run_ours(args, world, rank, local):
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # the attention kernel at each shift of the cycle alone (window types differ per shift)
+    per_shift = {}
+    for i, e in enumerate(evs):
+        per_shift.setdefault(str(tuple(shifts[i % len(shifts)])), []).append(e[2].elapsed_time(e[3]))
+    per_shift_ms = {k: round(statistics.mean(v), 4) for k, v in per_shift.items()}
 
     flops = cnt["attn_flops"]
     value = world * flops / (step_ms * 1e-3) / 1e12
@@ -249,6 +254,12 @@ def run_ours(args, world, rank, local):
             "parallelism": f"(batch, head) units sharded over {world} GPU(s), {wl.B * wl.heads} per GPU, no data-path collective",
             "l2": f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush",
         },
+        "dense_equivalent": {
+            "note": "context only: the dense attention this layer replaces, at the measured step time",
+            "sparsity": round(accounting.sparsity(cnt["keys_per_query"], wl.N + wl.n_text), 4),
+            "tflops": round(world * accounting.dense_attn_flops(wl.B, wl.heads, wl.N, wl.d, wl.N + wl.n_text)
+                            / (step_ms * 1e-3) / 1e12, 1),
+        },
         "pct_of_peak": {
             "step_vs_measured_burst": round(value / world / peak, 4),
             "step_vs_nominal_2250": round(value / world / 2250.0, 4),
@@ -263,6 +274,7 @@ def run_ours(args, world, rank, local):
             "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 1.59 PF/s",
             "traffic": traffic,
             "attn_ms": round(attn_ms, 4),
+            "attn_ms_per_shift": per_shift_ms,
         },
         "hbm_kernels": hbm_lines(cnt, pool_ms, route_ms, peaks["hbm_gbs"], fused),
         "clocks": clocks,
