@@ -316,7 +316,7 @@ def run_text_queries(args, layer, wl, kd, vd):
     achieved = flops / (ms * 1e-3) / 1e12
     return {"ms": round(ms, 4), "gflop": round(flops / 1e9, 2), "value": round(achieved, 2), "unit": "TFLOP/s",
             "frac_of_measured_bf16": round(achieved / peaks["bf16_tflops"], 4),
-            "workspace_bytes": layer.text_workspace.numel() if getattr(layer, "text_workspace", None) is not None else 0}
+            "workspace_bytes": layer.text_workspace.numel() if layer.text_workspace is not None else 0}
 
 
 def run_backward(args):

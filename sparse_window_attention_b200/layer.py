@@ -42,6 +42,8 @@ class BasaLayer:
         # its workspace size depends on the shift and grows on first use
         self.fused = self.has_pool and routed_k > 0
         self.fused_workspace = None
+        self.text_workspace = None  # text-query rows: per-split partial results
+        self._branch_bufs = []      # branch form: (out, lse) per branch
 
     def params(self, shift, **extra) -> B.basa_params:
         key = (tuple(shift), tuple(sorted(extra.items())))
@@ -98,7 +100,7 @@ class BasaLayer:
                 self.pool_kv(k, v, shift, stream)
             if self.routed_k > 0:
                 self.route(q, k, shift, stream)
-        if not hasattr(self, "_branch_bufs") or len(self._branch_bufs) < len(splits):
+        if len(self._branch_bufs) < len(splits):
             self._branch_bufs = [(torch.empty_like(q), torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device))
                                  for _ in splits]
         for (o, l), keys in zip(self._branch_bufs, splits):
@@ -112,7 +114,7 @@ class BasaLayer:
         nbytes = B.basa_text_attn_workspace_bytes(self.params((0, 0, 0)))
         ws = None
         if nbytes > 0:
-            if getattr(self, "text_workspace", None) is None or self.text_workspace.numel() < nbytes:
+            if self.text_workspace is None or self.text_workspace.numel() < nbytes:
                 self.text_workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
             ws = self.text_workspace
         B.basa_text_attn_fwd(q_text, k, v, out_text, ws, self.params((0, 0, 0)), stream)
