@@ -244,16 +244,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {
-            "workload": f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} grid={'x'.join(map(str, wl.grid))} "
-                        f"window={'x'.join(map(str, wl.window))} shifts={shifts} pool={'x'.join(map(str, wl.pool))} "
-                        f"text={wl.n_text} routed_k={wl.routed_k}"
-                        + (f" route_radius={wl.route_radius}" if wl.route_radius else ""),
-            "keys_per_query": cnt["keys_per_query"],
-            "attn_gflop_per_layer": round(flops / 1e9, 2),
-            "parallelism": f"(batch, head) units sharded over {world} GPU(s), {wl.B * wl.heads} per GPU, no data-path collective",
-            "l2": f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush",
-        },
+        "config": workload_config(wl, world),
         "dense_equivalent": {
             "note": "context only: the dense attention this layer replaces, at the measured step time",
             "sparsity": round(accounting.sparsity(cnt["keys_per_query"], wl.N + wl.n_text), 4),
@@ -383,6 +374,23 @@ def run_branch_form(args, layer, qd, kd, vd, shifts, flops):
     return {"splits": "windows | pooled + text", "ms_per_step": round(ms, 4),
             "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "launches_per_step": layer.launches_per_forward() + len(splits)}
+
+
+def workload_config(wl, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    cnt = accounting.workload_counts(wl)
+    shifts = synth.SHIFT_CYCLES[wl.name]
+    return {
+        "workload": f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} grid={'x'.join(map(str, wl.grid))} "
+                    f"window={'x'.join(map(str, wl.window))} shifts={shifts} pool={'x'.join(map(str, wl.pool))} "
+                    f"text={wl.n_text} routed_k={wl.routed_k}"
+                    + (f" route_radius={wl.route_radius}" if wl.route_radius else ""),
+        "keys_per_query": cnt["keys_per_query"],
+        "attn_gflop_per_layer": round(cnt["attn_flops"] / 1e9, 2),
+        "parallelism": f"(batch, head) units sharded over {world} GPU(s), {wl.B * wl.heads} per GPU, "
+                       "no data-path collective",
+        "l2": f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush",
+    }
 
 
 def hbm_lines(cnt, pool_ms, route_ms, hbm_gbs, fused):
@@ -532,7 +540,7 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "keys_per_query": cnt["keys_per_query"]},
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(tflops, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
