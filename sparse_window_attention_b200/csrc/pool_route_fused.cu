@@ -67,7 +67,7 @@ struct CellCtrl {
 // Runs of the windows met by the box [o, o + e) along one axis (window extent w,
 // shift s, grid extent G): original coordinate c lies in window ((c - s) mod G) / w,
 // and window boundaries fall every w coordinates of the shifted axis.
-__device__ void build_runs(int o, int e, int w, int s, int G, AxisRun *runs, int *n_out) {
+__host__ __device__ void build_runs(int o, int e, int w, int s, int G, AxisRun *runs, int *n_out) {
   int n = 0;
   int c = 0;
   while (c < e && n < kMaxAxisRuns) {
@@ -88,7 +88,7 @@ __device__ void build_runs(int o, int e, int w, int s, int G, AxisRun *runs, int
 
 // Cells of one axis in coordinate order: the run intervals cut at pool-patch
 // boundaries (multiples of p).
-__device__ void build_cells(const AxisRun *runs, int n_runs, int p, AxisCell *cells, int *n_out) {
+__host__ __device__ void build_cells(const AxisRun *runs, int n_runs, int p, AxisCell *cells, int *n_out) {
   int n = 0;
   // intervals in coordinate order: run 0, 1, ..., n_runs - 1, then run 0's wrapped part
   for (int k = 0; k <= n_runs; ++k) {
