@@ -11,6 +11,15 @@
  *   basa_route_windows    top-k routed windows          (BASA §3.3, §A.2)
  *   basa_window_attn_fwd  shifted-window attention      (BASA §3.1, §A.1)
  *
+ * and further entry points serve the same layer:
+ *
+ *   basa_pool_route           the first two from one read of q, k, v
+ *   basa_route_windows_noalloc  routing without a caller workspace
+ *   basa_window_attn_fwd_lse  one branch of the decomposed form, with log-sum-exp
+ *   basa_merge_branches       branches merged into the joint softmax  (BASA §A.1)
+ *   basa_text_attn_fwd        the text queries' output rows (dense over all keys)
+ *   basa_window_attn_bwd      gradients w.r.t. q, k, v (float32)       (BASA §3.4)
+ *
  * Conventions common to every entry point
  * ---------------------------------------
  * Pointers. Every tensor pointer is a DEVICE pointer owned by the caller; the
@@ -36,8 +45,10 @@
  * Errors. Arguments are checked on the host before anything is launched; an
  *   invalid call returns an error code and launches nothing. A launch failure
  *   returns BASA_ERR_CUDA. No entry point aborts, traps or prints.
- * Threads. Entry points are reentrant; the only library state is the lazily
- *   resolved driver entry point used to encode TMA tensor maps.
+ * Threads. Entry points are reentrant. Library state: the lazily resolved
+ *   driver entry point used to encode TMA tensor maps, a mutex-guarded cache of
+ *   window tiling plans, per-device SM counts and kernel attributes set once,
+ *   and the scratch array of basa_route_windows_noalloc.
  */
 #ifndef BASA_H
 #define BASA_H
