@@ -24,7 +24,9 @@ blocking, fusion or reordering beyond what the definition needs:
 6. inverse shift of the output.
 
 The branch form (branch_attention, merge_branches) evaluates key groups separately
-with their log-sum-exp and merges them (BASA §A.1).
+with their log-sum-exp and merges them (BASA §A.1). text_query_attention gives the
+text queries' rows (dense over every key), and basa_attention_backward the
+gradients of basa_attention with respect to q, k and v (routing held fixed).
 
 Readings taken where the pages are silent:
   * shift convention Xr[t,y,x] = X[(t+st)%T, (y+sy)%H, (x+sx)%W] (roll by -s);
