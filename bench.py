@@ -278,7 +278,7 @@ def run_ours(args, world, rank, local):
         if wl.n_text > 0:
             res["text_queries"] = run_text_queries(args, layer, wl, kd, vd)
         res["backward_f32"] = run_backward(args)
-        for name in ("wan", "wan_video"):
+        for name in ("wan", "wan_video", "flux1k", "flux4k"):
             if args.workload != name:
                 res["also_" + name] = run_also(args, name)
     return res
@@ -473,8 +473,8 @@ def run_e2e(args, layer, q, k, v, shifts, flops, world):
 
 def run_also(args, name):
     """Secondary workload on the same GPU (context for the headline line)."""
-    # about a second of timed work each: a video layer is ~50x a FLUX-2K layer
-    steps = max(10, args.steps // 50) if name == "wan_video" else max(50, args.steps // 4)
+    # about a second of timed work each: a video layer is ~50x a FLUX-2K layer, FLUX-4K ~4x
+    steps = {"wan_video": max(10, args.steps // 50), "flux4k": max(20, args.steps // 16)}.get(name, max(50, args.steps // 4))
     sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True, "steps": steps})
     r = run_ours(sub, 1, 0, int(os.environ.get("LOCAL_RANK", "0")))
     return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "hbm_kernels", "gpu_launches")}
