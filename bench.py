@@ -5,9 +5,15 @@
 
 A step is one layer call over one batch of synthetic inputs already resident in
 HBM; consecutive steps walk the workload's shift cycle (one shift per layer).
-Rank 0 prints ONE JSON line. Multi-GPU runs (torchrun) give every rank its own
-copy of the workload (the path shards over (batch, head) with no exchange),
-time on the device and report the max over ranks ("scaling": "weak").
+Rank 0 prints ONE JSON line. Multi-GPU runs (torchrun) time on the device and
+report the max over ranks; by default every rank runs its own full copy of the
+workload ("scaling": "weak"); with `--shard heads` one layer's (batch, head)
+units are split over the ranks ("scaling": "strong"). Either way there is no
+exchange on the data path: pooling, routing and attention have no term across heads.
+
+L2: workloads whose inputs exceed the 126 MB L2 are timed back to back; for
+smaller ones the line adds `l2_flushed`, every step timed after a 256 MB scratch
+write outside the events.
 
 The line also carries: `roofline` (the attention kernel's achieved TFLOP/s from
 CUDA events around its launches, against the measured bf16 peak, and its DRAM
@@ -45,6 +51,7 @@ from sparse_window_attention_b200 import accounting, sharding, synth  # noqa: E4
 
 METRIC = "shifted-window attn fwd effective TFLOP/s & % of B200 BF16 peak; ms/layer"
 ATTN_SOURCE = os.path.join(ROOT, "sparse_window_attention_b200", "csrc", "attn_bf16_sm100.cu")
+L2_BYTES = 126e6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -72,17 +79,57 @@ def kernel_traffic(kernel_file: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and throttle reasons sampled DURING the timed region.
 
+    NVML is polled from a thread every ~0.5 ms (a timed region of a few ms still
+    gets samples); without NVML, `nvidia-smi -lms 100` is the fallback."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.stop = threading.Event()
+        self.samples = []  # (sm_mhz, reason bits)
+        self.max_mhz = None
         self.lines = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:  # the device torch uses, whatever CUDA_VISIBLE_DEVICES says
+            pr = torch.cuda.get_device_properties(self.index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def __enter__(self):
         try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml, every 0.5 ms"
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                             int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        break
+                    time.sleep(0.0005)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            pass
+        try:
+            self.source = "nvidia-smi -lms 100"
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100", "-i", str(self.index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
@@ -90,6 +137,7 @@ class ClockSampler:
             self.thread.start()
         except (FileNotFoundError, OSError):
             self.proc = None
+            self.source = None
         return self
 
     def _read(self):
@@ -97,17 +145,20 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if getattr(self, "thread", None) is not None:
             self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [s for s, _ in self.samples], self.max_mhz, set()
+        for _, bits in self.samples:
+            reasons.update(n for n, b in self.REASONS if bits & b)
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
@@ -117,12 +168,12 @@ class ClockSampler:
                 mx = float(parts[1])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[3:7]):
+            for (n, _), v in zip(self.REASONS, parts[3:7]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm), "source": self.source}
+        return out
 
 
 def dist_setup():
@@ -161,10 +212,21 @@ def run_ours(args, world, rank, local):
     wl = synth.WORKLOADS[args.workload]
     cnt = accounting.workload_counts(wl)
     shifts = synth.SHIFT_CYCLES[args.workload]
-    q, k, v = synth.make_inputs(wl, seed=args.seed + rank)
+    strong = getattr(args, "shard", "replicas") == "heads"
+    if strong:
+        # one layer split over the ranks by (batch, head) units: every rank draws the
+        # same full inputs and keeps its own units (no exchange on the data path)
+        layer = BasaLayer.for_shard(wl.B, wl.heads, wl.d, wl.grid, wl.window, world, rank, pool=wl.pool,
+                                    n_text=wl.n_text, routed_k=wl.routed_k, dtype=wl.dtype,
+                                    route_radius=wl.route_radius)
+        q, k, v = (layer.shard_of(x).contiguous() for x in synth.make_inputs(wl, seed=args.seed))
+        unit_frac = (layer.units[1] - layer.units[0]) / (wl.B * wl.heads)
+    else:
+        q, k, v = synth.make_inputs(wl, seed=args.seed + rank)
+        layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
+                          route_radius=wl.route_radius)
+        unit_frac = 1.0
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
-    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
-                      route_radius=wl.route_radius)
     out = torch.empty_like(qd)
     stream = torch.cuda.current_stream()
 
@@ -215,6 +277,32 @@ def run_ours(args, world, rank, local):
     for i in range(n_ev):
         step(i, evs[i])
     torch.cuda.synchronize()
+    l2_flushed = None
+    if cnt["attn_bytes"] < L2_BYTES:
+        # the inputs fit in L2: also time every step after a 256 MB scratch write
+        # (outside the events), which evicts them, so the kernels read from HBM
+        scratch = torch.empty(256 << 20, dtype=torch.uint8, device=qd.device)
+        fevs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n_ev)]
+        for i in range(n_ev):
+            scratch.fill_(i & 0xFF)
+            step(i, fevs[i])
+        torch.cuda.synchronize()
+        del scratch
+        f_step = statistics.mean(e[0].elapsed_time(e[3]) for e in fevs)
+        f_attn = statistics.mean(e[2].elapsed_time(e[3]) for e in fevs)
+        f_pool = statistics.mean(e[0].elapsed_time(e[1]) for e in fevs)
+        f_route = statistics.mean(e[1].elapsed_time(e[2]) for e in fevs)
+        f_ach = cnt["attn_flops"] / (f_attn * 1e-3) / 1e12
+        peaks0, _ = load_peaks()
+        l2_flushed = {
+            "how": "256 MB scratch write before every step, outside the CUDA events; step = pool start to attention end",
+            "steps": n_ev,
+            "ms_per_step": round(f_step, 4),
+            "value": round(cnt["attn_flops"] / (f_step * 1e-3) / 1e12, 2),
+            "attn_ms": round(f_attn, 4),
+            "attn_frac_of_measured_bf16": round(f_ach / peaks0["bf16_tflops"], 4),
+            "hbm_kernels": hbm_lines(cnt, f_pool, f_route, peaks0["hbm_gbs"], fused),
+        }
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -225,10 +313,12 @@ def run_ours(args, world, rank, local):
     per_shift_ms = {k: round(statistics.mean(v), 4) for k, v in per_shift.items()}
 
     flops = cnt["attn_flops"]
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    # whole-job throughput: the full layer split over the ranks (strong) or one
+    # full layer per rank (weak); the per-rank kernel does unit_frac of a layer
+    value = (1 if strong else world) * flops / (step_ms * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
     peak = peaks["bf16_tflops"]
-    achieved = flops / (attn_ms * 1e-3) / 1e12
+    achieved = unit_frac * flops / (attn_ms * 1e-3) / 1e12
     traffic = kernel_traffic(ATTN_SOURCE, args.workload)
     clocks = sampler.summary()
     res = {
@@ -240,11 +330,11 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if strong else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": workload_config(wl, world),
+        "config": workload_config(wl, world, strong),
         "dense_equivalent": {
             "note": "context only: the dense attention this layer replaces, at the measured step time",
             "sparsity": round(accounting.sparsity(cnt["keys_per_query"], wl.N + wl.n_text), 4),
@@ -254,6 +344,7 @@ def run_ours(args, world, rank, local):
         "pct_of_peak": {
             "step_vs_measured_burst": round(value / world / peak, 4),
             "step_vs_nominal_2250": round(value / world / 2250.0, 4),
+            "attn_kernel_vs_nominal_2250": round(achieved / 2250.0, 4),
         },
         "roofline": {
             "kernel": "attn_bf16_kernel",
@@ -269,10 +360,11 @@ def run_ours(args, world, rank, local):
         },
         "hbm_kernels": hbm_lines(cnt, pool_ms, route_ms, peaks["hbm_gbs"], fused),
         "clocks": clocks,
+        "l2_flushed": l2_flushed,
         "gpu_launches": args.steps * layer.launches_per_forward(),
     }
     if not args.no_e2e:
-        res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world)
+        res["e2e"] = run_e2e(args, layer, q, k, v, shifts, flops, world, 1 if strong else world)
     if not args.no_extra and world == 1:
         res["branch_form"] = run_branch_form(args, layer, qd, kd, vd, shifts, flops)
         if wl.n_text > 0:
@@ -376,7 +468,7 @@ def run_branch_form(args, layer, qd, kd, vd, shifts, flops):
             "launches_per_step": layer.launches_per_forward() + len(splits)}
 
 
-def workload_config(wl, world):
+def workload_config(wl, world, strong=False):
     """The `config` object of the JSON line (the same for both arms)."""
     cnt = accounting.workload_counts(wl)
     shifts = synth.SHIFT_CYCLES[wl.name]
@@ -387,9 +479,13 @@ def workload_config(wl, world):
                     + (f" route_radius={wl.route_radius}" if wl.route_radius else ""),
         "keys_per_query": cnt["keys_per_query"],
         "attn_gflop_per_layer": round(cnt["attn_flops"] / 1e9, 2),
-        "parallelism": f"(batch, head) units sharded over {world} GPU(s), {wl.B * wl.heads} per GPU, "
-                       "no data-path collective",
-        "l2": f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush",
+        "parallelism": (f"one layer's {wl.B * wl.heads} (batch, head) units split over {world} GPU(s) "
+                        "(sharding.unit_shard), no data-path collective" if strong else
+                        f"replicas: a full layer ({wl.B * wl.heads} (batch, head) units) per GPU on each of "
+                        f"{world} GPU(s), no data-path collective"),
+        "l2": (f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB > 126 MB L2; no flush" if cnt["attn_bytes"] >= L2_BYTES else
+               f"inputs {cnt['attn_bytes'] / 1e6:.0f} MB < 126 MB L2: the headline times back-to-back steps (warm "
+               "L2); `l2_flushed` times every step after a 256 MB scratch write"),
     }
 
 
@@ -410,13 +506,14 @@ def hbm_lines(cnt, pool_ms, route_ms, hbm_gbs, fused):
             "route": line(route_ms, cnt["route_bytes"], "box means over windows, top-k")}
 
 
-def run_e2e(args, layer, q, k, v, shifts, flops, world):
+def run_e2e(args, layer, q, k, v, shifts, flops, world, job_layers=None):
     """Same metric through the public API with host (pinned) buffers: every step
     copies its q, k, v host->device, runs the layer and copies the output back.
     Steps are pipelined over three streams with two device buffer sets: the inputs
     of step i + 1 travel host->device while step i computes and step i - 1's output
     travels device->host (PCIe is full duplex); every step's copies are inside the
     timed region, which runs from the first input copy to the last output copy."""
+    job_layers = world if job_layers is None else job_layers  # full layers the job computes per step
     hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     hout = torch.empty_like(hq).pin_memory()
     sets = [tuple(torch.empty_like(x, device="cuda") for x in (hq, hk, hv)) for _ in range(2)]
@@ -461,7 +558,7 @@ def run_e2e(args, layer, q, k, v, shifts, flops, world):
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
     esz = hq.element_size()
     return {
-        "value": round(world * flops / (ms * 1e-3) / 1e12, 2),
+        "value": round(job_layers * flops / (ms * 1e-3) / 1e12, 2),
         "unit": "TFLOP/s",
         "ms_per_step": round(ms, 3),
         "steps": steps,
@@ -477,7 +574,8 @@ def run_also(args, name):
     steps = {"wan_video": max(10, args.steps // 50), "flux4k": max(20, args.steps // 16)}.get(name, max(50, args.steps // 4))
     sub = argparse.Namespace(**{**vars(args), "workload": name, "no_e2e": True, "no_extra": True, "steps": steps})
     r = run_ours(sub, 1, 0, int(os.environ.get("LOCAL_RANK", "0")))
-    return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "hbm_kernels", "gpu_launches")}
+    return {k: r[k] for k in ("value", "ms_per_step", "config", "roofline", "hbm_kernels", "gpu_launches",
+                               "l2_flushed") if r.get(k) is not None}
 
 
 # ----------------------------------------------------------------- oracle (CPU)
@@ -516,6 +614,42 @@ def cpu_oracle_sample(wl, budget_s: float, max_units: int | None = None):
     return units * flops_per_unit / el / 1e12, units, el, threads
 
 
+def host_cpu():
+    """(logical CPUs this process may use, CPU model name)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return n, model
+
+
+def cpu_baseline(args):
+    """The oracle on the host: one BLAS thread, then all of them (numpy's pool)."""
+    from threadpoolctl import threadpool_limits
+
+    wl = synth.WORKLOADS[args.workload]
+    nproc, model = host_cpu()
+    with threadpool_limits(limits=1):
+        t1, u1, e1, _ = cpu_oracle_sample(wl, args.cpu_budget / 3)
+    tn, un, en, threads = cpu_oracle_sample(wl, args.cpu_budget)
+    return {
+        "value": round(tn, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+        "single_thread_value": round(t1, 6),
+        "nproc": nproc, "cpu_model": model,
+        "sample": f"{un} (head, window) units of {args.workload}, head 0, {en:.1f} s on {threads} BLAS threads "
+                  f"(single thread: {u1} units, {e1:.1f} s), float64 numpy",
+    }
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return None
@@ -541,7 +675,8 @@ def run_reference(args, world, rank):
         "dtype": "f64",
         "data": "synthetic",
         "config": workload_config(wl, world),
-        "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample,
+                         "nproc": host_cpu()[0], "cpu_model": host_cpu()[1]},
         "e2e": {"value": round(tflops, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -553,6 +688,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="flux2k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: a full layer per GPU (weak scaling); heads: one layer's (batch, head) units "
+                         "split over the GPUs (strong scaling)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
@@ -573,11 +711,7 @@ def main():
     world, rank, local = dist_setup()
     res = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu:
-        tflops, units, el, threads = cpu_oracle_sample(synth.WORKLOADS[args.workload], args.cpu_budget)
-        res["cpu_baseline"] = {
-            "value": round(tflops, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{units} (head, window) units of {args.workload}, head 0, {el:.1f} s, float64 numpy",
-        }
+        res["cpu_baseline"] = cpu_baseline(args)
     if world > 1:
         import torch.distributed as dist
 

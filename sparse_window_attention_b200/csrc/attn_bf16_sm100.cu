@@ -51,8 +51,7 @@ constexpr int kMaskTable = 64;                         // key tiles whose column
 constexpr uint32_t kSmemMask = kSmemCtrl + kCtrlBytes;
 constexpr uint32_t kSmemBytes = kSmemMask + kMaskTable * 16 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr int kDefaultEmuPairs = 0;
-constexpr int kMaxTextSplits = 8;  // key-range splits of the text-query rows  // exponential pairs of every 8 done on the FMA pipe
+constexpr int kMaxTextSplits = 8;  // key-range splits of the text-query rows
 
 // tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), N >> 3 at bits 17-22, M >> 4 at bits 24-28; bit 16 marks
@@ -235,32 +234,12 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 // produced, which float32 sums and bfloat16 P hold exactly as well. This skips
 // most rescales of the O accumulator in TMEM.
 constexpr float kRescaleLog2 = 8.0f;
-// 2^f on [-1/2, 1/2]: degree-3 polynomial minimising the maximum relative error
-// (Remez exchange fitted for this kernel; max relative error 7.5e-5, far below
-// the 2^-9 rounding of the bfloat16 P that consumes it).
-constexpr float kExpC0 = 0.9999280571937561f;
-constexpr float kExpC1 = 0.6932609677314758f;
-constexpr float kExpC2 = 0.2426111251115799f;
-constexpr float kExpC3 = 0.0551716685295105f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer in the low mantissa bits
-
-// Which pairs of every 8 take the FMA-pipe exponential, spread evenly so the
-// emulated pairs interleave with MUFU ones: bit k set = pair k (mod 8) emulated.
-__host__ __device__ constexpr uint32_t emu_pair_mask(int n) {
-  return n <= 0 ? 0x00u : n == 1 ? 0x80u : n == 2 ? 0x88u : n == 3 ? 0xA4u : 0xAAu;
-}
-
-// P = 2^x (x = s * scale_log2 - m) for the 128 scores of a row, written in place as
-// the 64 bfloat16 pairs the P V MMA reads (s[i] = pair (2i, 2i+1), low half = even
-// key); each pair is packed as soon as it is computed, so the live register set
-// shrinks along the row. Returns the float32 row sum. For the pairs selected by
-// emu_pair_mask(EMU_PAIRS) the exponential runs on the FMA pipe (x = j + f with
-// j = round(x), 2^f by the polynomial, 2^j added to the exponent bits), the rest
-// on the MUFU ex2 unit.
-template <int EMU_PAIRS>
+// P = 2^x (x = s * scale_log2 - m) for the 128 scores of a row (MUFU ex2), written
+// in place as the 64 bfloat16 pairs the P V MMA reads (s[i] = pair (2i, 2i+1), low
+// half = even key); each pair is packed as soon as it is computed, so the live
+// register set shrinks along the row. Returns the float32 row sum.
 __device__ __forceinline__ float exp2_row_packed(uint32_t (&s)[128], float scale_log2, float m) {
   using namespace ptx;
-  constexpr uint32_t kEmu = emu_pair_mask(EMU_PAIRS);
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2), negm2 = f2_pack(-m, -m);
   uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
@@ -268,27 +247,11 @@ __device__ __forceinline__ float exp2_row_packed(uint32_t (&s)[128], float scale
     const uint64_t x = ffma2(f2_pack(__uint_as_float(s[2 * pr]), __uint_as_float(s[2 * pr + 1])), sc2, negm2);
     float x0, x1;
     f2_unpack(x, x0, x1);
-    uint32_t r0, r1;
-    if ((kEmu >> (pr & 7)) & 1u) {
-      const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-      const uint64_t t = fadd2(xc, f2_pack(kRoundMagic, kRoundMagic));
-      const uint64_t f = ffma2(fadd2(t, f2_pack(-kRoundMagic, -kRoundMagic)), f2_pack(-1.f, -1.f), xc);
-      uint64_t q = ffma2(f, f2_pack(kExpC3, kExpC3), f2_pack(kExpC2, kExpC2));
-      q = ffma2(q, f, f2_pack(kExpC1, kExpC1));
-      q = ffma2(q, f, f2_pack(kExpC0, kExpC0));
-      float q0, q1, t0, t1;
-      f2_unpack(q, q0, q1);
-      f2_unpack(t, t0, t1);
-      r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
-      r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
-    } else {
-      r0 = __float_as_uint(ex2(x0));
-      r1 = __float_as_uint(ex2(x1));
-    }
-    const uint64_t pp = f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+    const float r0 = ex2(x0), r1 = ex2(x1);
+    const uint64_t pp = f2_pack(r0, r1);
     if (pr & 1) acc1 = fadd2(acc1, pp);
     else acc0 = fadd2(acc0, pp);
-    s[pr] = pack_bf16x2(__uint_as_float(r0), __uint_as_float(r1));  // s[pr] was read at pair pr / 2
+    s[pr] = pack_bf16x2(r0, r1);  // s[pr] was read at pair pr / 2
   }
   float a, b, c, d;
   f2_unpack(acc0, a, b);
@@ -324,7 +287,6 @@ __device__ __forceinline__ void apply_mask(uint32_t (&s)[N], const uint32_t *mas
   }
 }
 
-template <int EMU_PAIRS>
 __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -562,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       const bool need = m_tile > m + kRescaleLog2;  // always true on the first tile (m = -inf)
       const float m_new = need ? m_tile : m;
       const float alpha = need ? ptx::ex2(m - m_new) : 1.0f;
-      const float sum = exp2_row_packed<EMU_PAIRS>(s, sl2, m_new);
+      const float sum = exp2_row_packed(s, sl2, m_new);
       l = l * alpha + sum;
       m = m_new;
       // P row -> TMEM over the first 64 columns of S; the MMA that overwrites S
@@ -704,18 +666,9 @@ bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, lon
 }
 
 basa_status run_attn(const AttnParams &P, long long blocks, cudaStream_t s) {
-  static const int emu = [] {
-    // tuning override for the share of exponentials done on the FMA pipe (pairs of 8)
-    const char *e = std::getenv("BASA_TUNE_EXP_EMU");
-    const int v = e ? std::atoi(e) : kDefaultEmuPairs;
-    return (v == 0 || v == 2) ? v : kDefaultEmuPairs;
-  }();
-  // Measured on B200 (FLUX 2048^2): every share of FMA-pipe exponentials tried (1/8 to 1/2)
-  // was slower than MUFU only, so 0 is the default; the variant stays for other parts/shapes.
-  auto kernel = emu == 2 ? attn_bf16_kernel<2> : attn_bf16_kernel<0>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return BASA_ERR_CUDA;
-  kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
+  attn_bf16_kernel<<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 

@@ -14,6 +14,7 @@
 #include <cfloat>
 #include <climits>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "basa_internal.h"
@@ -324,14 +325,16 @@ basa_status launch_topk(const float *qm, const float *km, int32_t *route_idx, fl
   const int bh = p.B * p.heads;
   RouteArgs r{qm, km, route_idx, route_score, g.nWin, p.head_dim, p.routed_k, p.route_radius, g.nWy, g.nWx};
   const size_t smem = (size_t(kRouteChunk) * (p.head_dim + 4) + kRouteWarps * p.head_dim + size_t(kRouteWarps) * g.nWin) * sizeof(float);
-  static std::once_flag once_wide[64];
+  // The shared-memory limit is raised once per device; a failed attempt is not
+  // recorded, so every later call retries it and reports its own error.
+  static std::atomic<int> wide_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BASA_ERR_CUDA;
-  cudaError_t e = cudaSuccess;
-  std::call_once(once_wide[dev], [&] {
-    e = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  });
-  if (e != cudaSuccess) return BASA_ERR_CUDA;
+  if (!wide_set[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+      return BASA_ERR_CUDA;
+    wide_set[dev].store(1, std::memory_order_release);
+  }
   const int ngroups = (g.nWin + kRouteWarps - 1) / kRouteWarps;
   route_topk_kernel<<<unsigned(bh) * unsigned(ngroups), kRouteWarps * 32, smem, s>>>(r);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;

@@ -10,6 +10,7 @@ from __future__ import annotations
 import torch
 
 from . import binding as B
+from . import sharding
 
 
 class BasaLayer:
@@ -44,6 +45,22 @@ class BasaLayer:
         self.fused_workspace = None
         self.text_workspace = None  # text-query rows: per-split partial results
         self._branch_bufs = []      # branch form: (out, lse) per branch
+
+    @classmethod
+    def for_shard(cls, batch, heads, head_dim, grid, window, world, rank, **kw):
+        """The layer for rank `rank` of `world` GPUs splitting the (batch, head) units
+        (sharding.unit_shard): it runs B = 1 and its own units as heads, on the views
+        `layer.shard_of(x)` of the full tensors. Pooling, routing and attention have no
+        term across heads, so the shards need no exchange."""
+        start, stop = sharding.unit_shard(batch, heads, world, rank)
+        layer = cls(1, stop - start, head_dim, grid, window, **kw)
+        layer.units = (start, stop)
+        return layer
+
+    def shard_of(self, x):
+        """This layer's units of a full [B, heads, rows, d] tensor (a view, no copy)."""
+        start, stop = getattr(self, "units", (0, self.batch * self.heads))
+        return sharding.shard_view(x, start, stop)
 
     def params(self, shift, **extra) -> B.basa_params:
         key = (tuple(shift), tuple(sorted(extra.items())))

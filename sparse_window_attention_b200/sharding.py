@@ -23,6 +23,17 @@ def unit_shard(B: int, heads: int, world: int, rank: int) -> tuple:
     return start, start + base + (1 if rank < extra else 0)
 
 
+def shard_view(x, start: int, stop: int):
+    """The units [start, stop) of a [B, heads, rows, d] tensor as a [1, stop - start,
+    rows, d] view of the same memory (no copy): with B and heads flattened, a range of
+    units is one contiguous block, so a layer built for B = 1 and stop - start heads
+    runs on it unchanged and writes its outputs in place."""
+    flat = x.reshape(1, -1, *x.shape[2:])
+    if flat.data_ptr() != x.data_ptr():
+        raise ValueError("shard_view needs a contiguous tensor")
+    return flat[:, start:stop]
+
+
 def max_over_ranks(value: float, group=None) -> float:
     """Max of a per-rank scalar over the process group (identity without one)."""
     import torch

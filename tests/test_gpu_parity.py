@@ -310,3 +310,39 @@ def test_repeat_calls_are_deterministic():
     b = layer.forward(qd, kd, vd, (0, 8, 8))
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------- every head of a full-size workload
+
+
+@pytest.mark.parametrize("name,shift", [("wan", (0, 3, 6)), ("flux2k", (0, 16, 16))])
+def test_every_head_full_size(name, shift):
+    """Pooling and routing compared on EVERY head of a full-size workload, and the
+    attention on sampled query rows of every head (a bug tied to the (batch, head)
+    index, e.g. a middle head's route-id or tensor-map offset, shows up here)."""
+    wl = synth.WORKLOADS[name]
+    (q, k, v), (qd, kd, vd) = PT.gpu_inputs(wl, 0)
+    geo = PT.geometry(wl, shift)
+    layer = _layer(wl)
+    out = layer.forward(qd, kd, vd, shift)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    rng = np.random.default_rng(5)
+    win = O.window_of_token(geo)
+    for h in range(wl.heads):
+        q64, k64, v64 = PT.to64(q[:, h:h + 1]), PT.to64(k[:, h:h + 1]), PT.to64(v[:, h:h + 1])
+        kp_ex, vp_ex = O.pool_kv(k64, v64, geo)
+        PT.assert_pool_close(PT.to64(layer.kp[:, h:h + 1]), kp_ex, wl.dtype)
+        PT.assert_pool_close(PT.to64(layer.vp[:, h:h + 1]), vp_ex, wl.dtype)
+        route = None
+        if geo.routed_k:
+            route, S = O.route_windows(q64, k64, geo)
+            assert PT.check_routes(layer.route_idx[:, h:h + 1].cpu().numpy(), route, S) == 0, f"head {h}"
+        # the kernel's own pooled K/V and routes, widened, are the oracle's inputs here:
+        # this checks the attention of head h, given what the earlier kernels produced
+        kp_g = PT.to64(layer.kp[:, h:h + 1])
+        vp_g = PT.to64(layer.vp[:, h:h + 1])
+        rows = np.unique(np.concatenate([rng.choice(wl.N, size=24, replace=False),
+                                         [np.nonzero(win == rng.integers(geo.n_win))[0][-1]]]))
+        ref = O.attention_rows(q64, k64, v64, geo, 0, 0, rows, kp=kp_g, vp=vp_g, route_idx=route)
+        PT.assert_outputs_close(PT.to64(out[0, h][rows]), ref, wl.dtype, f"{name} head {h}")

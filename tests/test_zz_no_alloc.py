@@ -28,13 +28,18 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_twice():
+    """Calls in a row: the Wan shape (1.7 MiB of window means), then 24 heads of the
+    same grid (3.4 MiB, most of the scratch array), then the Wan shape again with
+    other inputs, so the last call runs over stale means left past its own extent."""
     from sparse_window_attention_b200 import binding as B
 
-    wl = synth.WORKLOADS["wan"]
+    wan = synth.WORKLOADS["wan"]
+    wide = synth.Workload(**{**wan.__dict__, "name": "wan_24_heads", "heads": 24})
     nwin = 140
-    for call, seed in enumerate((0, 1)):
+    for call, (wl, seed) in enumerate(((wan, 0), (wide, 2), (wan, 1))):
         _, (qd, kd, _) = PT.gpu_inputs(wl, seed=seed)
         p = B.make_params(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.shift, wl.pool, wl.n_text, wl.routed_k, wl.dtype)
+        assert B.basa_route_workspace_bytes(p) <= 4 << 20
         shape = (wl.B, wl.heads, nwin, wl.routed_k)
         idx_ws = torch.full(shape, -1, dtype=torch.int32, device="cuda")
         sc_ws = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
