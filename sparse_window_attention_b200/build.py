@@ -19,8 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbasa.so")
-SOURCES = ["api.cpp", "plan.cpp", "pool_route.cu", "pool_route_fused.cu", "merge.cu", "attn_f32.cu", "attn_bf16_sm100.cu"]
-HEADERS = [os.path.join(CSRC, h) for h in ("basa_internal.h", "sm100_ptx.cuh")] + [os.path.join(ROOT, "include", "basa.h")]
+SOURCES = ["api.cpp", "plan.cpp", "pool_route.cu", "pool_route_fused.cu", "merge.cu", "attn_f32.cu", "attn_bf16_sm100.cu", "attn_bwd_bf16_sm100.cu"]
+HEADERS = [os.path.join(CSRC, h) for h in ("basa_internal.h", "sm100_ptx.cuh", "attn_sm100_common.cuh")] + [os.path.join(ROOT, "include", "basa.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

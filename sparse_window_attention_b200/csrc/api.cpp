@@ -205,8 +205,8 @@ basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v,
 }
 
 size_t basa_window_attn_bwd_workspace_bytes(const basa_params *p) {
-  if (check_common(p) != BASA_OK) return 0;
-  return basa::attn_bwd_workspace(*p);
+  if (check_common(p) != BASA_OK || p->head_dim != 128) return 0;
+  return p->dtype == BASA_BF16 ? basa::attn_bwd_bf16_workspace(*p) : basa::attn_bwd_workspace(*p);
 }
 
 basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v, const void *kp, const void *vp,
@@ -215,7 +215,9 @@ basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v, co
                                  basa_stream_t stream) {
   basa_status st = check_common(p);
   if (st != BASA_OK) return st;
-  if (p->dtype != BASA_F32 || p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (p->head_dim != 128) return BASA_ERR_UNSUPPORTED;
+  if (p->dtype == BASA_BF16 && p->routed_k > 0 && int64_t(p->T / p->wt) * (p->H / p->wh) * (p->W / p->ww) > 4096)
+    return BASA_ERR_UNSUPPORTED;
   if (empty_batch(p)) return BASA_OK;
   if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return BASA_ERR_INVALID_ARG;
   if (has_pool(p) != (kp != nullptr) || has_pool(p) != (vp != nullptr)) return BASA_ERR_INVALID_ARG;
@@ -225,9 +227,15 @@ basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v, co
     if (!aligned16(x)) return BASA_ERR_INVALID_ARG;
   if (!aligned4(lse) || (route_idx && !aligned4(route_idx))) return BASA_ERR_INVALID_ARG;
   if (kp && (!aligned16(kp) || !aligned16(vp))) return BASA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == BASA_BF16) {
+    const size_t need = basa::attn_bwd_bf16_workspace(*p);
+    if (need == 0) return BASA_ERR_UNSUPPORTED;  // the tiling plan does not fit the kernel's limits
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return BASA_ERR_INVALID_ARG;
+    return basa::launch_attn_bwd_bf16(q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv, workspace, *p, s);
+  }
   if (basa::attn_bwd_workspace(*p) > 0 && (!workspace || !aligned16(workspace))) return BASA_ERR_INVALID_ARG;
-  return basa::launch_attn_bwd_f32(q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv, workspace, *p,
-                                   reinterpret_cast<cudaStream_t>(stream));
+  return basa::launch_attn_bwd_f32(q, k, v, kp, vp, route_idx, out, lse, dout, dq, dk, dv, workspace, *p, s);
 }
 
 basa_status basa_merge_branches(int n, const void *const *outs, const float *const *lses, void *out, float *lse,

@@ -33,15 +33,20 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_sm100_common.cuh"
 #include "basa_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace basa {
 namespace {
 
+using sm100::kHalfBytes;
+using sm100::kTileBytes;
+using sm100::kTileDesc;
+using sm100::Waiter;
+using sm100::wrap;
+
 constexpr int kThreads = 320;  // 10 warps
-constexpr uint32_t kHalfBytes = 16384;                 // 128 rows x 128 B (64 bf16) , 128B-swizzled
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;        // 128 rows x head_dim 128
 constexpr int kStages = 5;
 constexpr uint32_t kSmemQ = 0;                         // 2 query tiles (reused for the output)
 constexpr uint32_t kSmemRing = 2 * kTileBytes;         // K/V ring
@@ -52,13 +57,6 @@ constexpr uint32_t kSmemMask = kSmemCtrl + kCtrlBytes;
 constexpr uint32_t kSmemBytes = kSmemMask + kMaskTable * 16 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxTextSplits = 8;  // key-range splits of the text-query rows
-
-// tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9, 10-12 = 1), N >> 3 at bits 17-22, M >> 4 at bits 24-28; bit 16 marks
-// B as MN-major (V is stored key-major with head_dim contiguous).
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);
-
 
 struct alignas(64) AttnParams {
   CUtensorMap map_q[kMaxShapes];
@@ -99,31 +97,6 @@ struct Ctrl {
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
-// Bounded mbarrier wait. Gives up when the shared abort flag is set or after
-// timeout_ns; the first waiter that times out sets the flag and its dev_err bit.
-struct Waiter {
-  Ctrl *c;
-  int32_t *dev_err;
-  unsigned long long limit;
-  int bit;
-  bool honor_abort;
-  __device__ bool wait(uint64_t *bar, uint32_t parity) const {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = ptx::globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (ptx::mbar_try_wait(bar, parity)) return true;
-      if ((it & 15u) == 0) {
-        if (honor_abort && *reinterpret_cast<volatile int *>(&c->abort)) return false;
-        if (ptx::globaltimer_ns() - t0 > limit) {
-          *reinterpret_cast<volatile int *>(&c->abort) = 1;
-          if (dev_err) atomicOr(dev_err, bit);
-          return false;
-        }
-      }
-    }
-  }
-};
-
 // Position in the key-tile stream: segments 0..routed_k are windows (own, then
 // routed), then the pooled tokens, then the text tokens.
 struct KeyIter {
@@ -150,29 +123,11 @@ __device__ __forceinline__ KeyIter first_key(const AttnParams &P, const Ctrl &c)
   return it;
 }
 
-__device__ __forceinline__ int wrap(int x, int g) { return x >= g ? x - g : x; }
-
-// Issue the TMA loads of one 128-row tile of a window (query, key or value tile).
-// Returns the bytes the loads will deliver.
-__device__ __forceinline__ uint32_t load_window_tile(const AttnParams &P, const CUtensorMap *maps, const PlanTile &tile,
-                                                     const int *org, int bh, uint8_t *dst, uint64_t *bar) {
-  uint32_t bytes = 0;
-  for (int i = 0; i < tile.n_pieces; ++i) {
-    const PlanPiece pc = P.plan.piece[tile.first_piece + i];
-    const int x = wrap(org[2] + pc.lx, P.g.W), y = wrap(org[1] + pc.ly, P.g.H), t = wrap(org[0] + pc.lt, P.g.T);
-    uint8_t *d = dst + uint32_t(pc.dest) * 128u;
-    ptx::tma_load_5d(d, &maps[pc.shape], bar, 0, x, y, t, bh);
-    ptx::tma_load_5d(d + kHalfBytes, &maps[pc.shape], bar, 64, x, y, t, bh);
-    bytes += uint32_t(P.plan.shape[pc.shape].rows) * 256u;
-  }
-  return bytes;
-}
-
 __device__ __forceinline__ uint32_t load_key_tile(const AttnParams &P, const Ctrl &c, const KeyIter &it, bool is_v,
                                                   int bh, uint8_t *dst, uint64_t *bar) {
   if (it.seg <= P.routed_k) {
     const PlanTile &tile = P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t];
-    return load_window_tile(P, is_v ? P.map_v : P.map_k, tile, c.org[it.seg], bh, dst, bar);
+    return sm100::load_window_tile(P.plan, P.g, is_v ? P.map_v : P.map_k, tile, c.org[it.seg], bh, dst, bar);
   }
   const bool pooled = it.seg == P.routed_k + 1;
   const CUtensorMap *map = pooled ? (is_v ? &P.map_vp : &P.map_kp) : (is_v ? &P.map_vt : &P.map_kt);
@@ -193,40 +148,8 @@ __device__ __forceinline__ bool key_tile_mask(const AttnParams &P, const Ctrl &c
   const bool pooled = it.seg == P.routed_k + 1;
   const int total = pooled ? P.n_pool : (P.dense ? P.dense_rows : P.n_text);
   const int valid = min(kTileRows, total - (pooled ? it.t : c.tile0 + it.t) * kTileRows);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int v = valid - 32 * i;
-    m[i] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
-  }
+  sm100::prefix_mask(valid, m);
   return valid == kTileRows;
-}
-
-// Shared-memory descriptors, split in 32-bit halves. The high half is constant:
-// stride byte offset 1024 (8 rows of 128 B), version 1, 128-byte swizzle. The
-// low half holds the start address >> 4 (bits 0-13) and the leading byte offset
-// (bits 16-29; ignored for K-major swizzled operands, 16 KB between the two
-// 64-column halves of the MN-major V). Stepping the start address is one add.
-constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-constexpr uint32_t kDescLoK = (16u >> 4) << 16;
-constexpr uint32_t kDescLoV = (kHalfBytes >> 4) << 16;
-
-// S (=) Q K^T over head_dim 128: 8 K-steps of 16; steps 0-3 walk the first 64-column
-// half in 32-byte strides, steps 4-7 the second half.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    ptx::mma_bf16_ss2(d_tmem, q_lo + off, kDescHi, k_lo + off, kDescHi, kIdescQK, kk > 0);
-  }
-}
-
-// O (+)= P V: P (bf16, 128 rows x 128 keys) sits in TMEM over the first 64
-// columns of its S buffer; 16 keys = 8 TMEM columns per K step.
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo, bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    ptx::mma_bf16_ts2(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
-                      (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // The running row max is only raised when a tile's max exceeds it by more than
@@ -363,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
   if (warp == 0) {
     // ------------------------------------------------------------- TMA loader
     if (lane == 0) {
-      Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, true};
-      Waiter drain{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
+      Waiter wt{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, true};
+      Waiter drain{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
       if (P.dense) {
         // whole 128-row boxes (rows past the end read as zero and still count)
         ptx::mbar_arrive_expect_tx(&c.q_full, (has_q1 ? 2u : 1u) * kTileBytes);
@@ -379,8 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
         if (has_q1) qbytes += uint32_t(P.plan.tile[ty.first_tile + q_tile0 + 1].valid_rows) * 256u;
         ptx::mbar_arrive_expect_tx(&c.q_full, qbytes);
         for (int g = 0; g < (has_q1 ? 2 : 1); ++g)
-          load_window_tile(P, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh,
-                           smem + kSmemQ + g * kTileBytes, &c.q_full);
+          sm100::load_window_tile(P.plan, P.g, P.map_q, P.plan.tile[ty.first_tile + q_tile0 + g], c.org[0], bh,
+                                  smem + kSmemQ + g * kTileBytes, &c.q_full);
       }
       KeyIter it = first_key(P, c);
       int last = -1;
@@ -415,20 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, true};
-      Waiter drain{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, false};
+      Waiter wt{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, true};
+      Waiter drain{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_MMA, false};
       // low descriptor halves of the query tiles and the ring slots
-      const uint32_t sQ = kDescLoK | (ptx::smem_u32(smem + kSmemQ) >> 4);
-      const uint32_t sRk = kDescLoK | (ptx::smem_u32(smem + kSmemRing) >> 4);
-      const uint32_t sRv = kDescLoV | (ptx::smem_u32(smem + kSmemRing) >> 4);
-      constexpr uint32_t kTileDesc = kTileBytes >> 4;
+      const uint32_t sQ = sm100::kDescLoK | (ptx::smem_u32(smem + kSmemQ) >> 4);
+      const uint32_t sRk = sm100::kDescLoK | (ptx::smem_u32(smem + kSmemRing) >> 4);
+      const uint32_t sRv = sm100::kDescLoMn | (ptx::smem_u32(smem + kSmemRing) >> 4);
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       if (wt.wait(&c.q_full, 0) && wt.wait(&c.full[0], 0)) {
         ptx::tc_fence_after();
-        issue_qk(tS0, sQ, sRk);
+        sm100::issue_ss(tS0, sQ, sRk);
         ptx::mma_commit(&c.s_full[0]);
         if (has_q1) {
-          issue_qk(tS1, sQ + kTileDesc, sRk);
+          sm100::issue_ss(tS1, sQ + kTileDesc, sRk);
           ptx::mma_commit(&c.s_full[1]);
         }
         ptx::mma_commit(&c.empty[0]);
@@ -439,11 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
           if (!wt.wait(&c.full[vi % kStages], (vi / kStages) & 1)) break;
           if (!wt.wait(&c.p_full[0], j & 1)) break;
           ptx::tc_fence_after();
-          issue_pv(tO0, tS0, vaddr, j > 0);
+          sm100::issue_ts(tO0, tS0, vaddr, j > 0);
           if (more) {
             if (!wt.wait(&c.full[ki % kStages], (ki / kStages) & 1)) break;
             ptx::tc_fence_after();
-            issue_qk(tS0, sQ, kaddr);
+            sm100::issue_ss(tS0, sQ, kaddr);
             ptx::mma_commit(&c.s_full[0]);
           } else {
             ptx::mma_commit(&c.o_full[0]);
@@ -451,12 +373,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
           if (has_q1) {
             if (!wt.wait(&c.p_full[1], j & 1)) break;
             ptx::tc_fence_after();
-            issue_pv(tO1, tS1, vaddr, j > 0);
+            sm100::issue_ts(tO1, tS1, vaddr, j > 0);
           }
           ptx::mma_commit(&c.empty[vi % kStages]);
           if (more) {
             if (has_q1) {
-              issue_qk(tS1, sQ + kTileDesc, kaddr);
+              sm100::issue_ss(tS1, sQ + kTileDesc, kaddr);
               ptx::mma_commit(&c.s_full[1]);
             }
             ptx::mma_commit(&c.empty[ki % kStages]);
@@ -479,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     const uint32_t lane_off = uint32_t(sub * 32) << 16;
     const uint32_t tS = tmem + lane_off + g * 128, tO = tmem + lane_off + 256 + g * 128;
     const bool active = g == 0 || has_q1;
-    Waiter wt{&c, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_SOFTMAX, true};
+    Waiter wt{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_SOFTMAX, true};
     uint8_t *q_tile = smem + kSmemQ + g * kTileBytes;
     const uint32_t swz = row & 7;
     const float sl2 = P.scale_log2;
@@ -594,16 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
         P.lse[((long long)split * P.bh_count + bh) * P.n_text + qrow] = (m + log2f(l)) * 0.6931471805599453f;
     } else if (ok && P.lse != nullptr) {
       // log-sum-exp of this row: m and l are in base 2 of the scaled scores
-      const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
-      for (int i = 0; i < tile.n_pieces; ++i) {
-        const PlanPiece pc = P.plan.piece[tile.first_piece + i];
-        const PlanShape sh = P.plan.shape[pc.shape];
-        const int local = row - int(pc.dest);
-        if (local < 0 || local >= sh.rows) continue;
-        const int lx = local % sh.cx, ly = (local / sh.cx) % sh.cy, lt = local / (sh.cx * sh.cy);
-        const int x = wrap(ox + pc.lx, P.g.W) + lx, y = wrap(oy + pc.ly, P.g.H) + ly, t = wrap(ot + pc.lt, P.g.T) + lt;
+      int t, y, x;
+      const int org[3] = {ot, oy, ox};
+      if (sm100::tile_row_token(P.plan, P.g, P.plan.tile[ty.first_tile + q_tile0 + g], org, row, &t, &y, &x))
         P.lse[(long long)bh * P.g.N + ((long long)t * P.g.H + y) * P.g.W + x] = (m + log2f(l)) * 0.6931471805599453f;
-      }
     }
     ptx::named_barrier(1 + g, 128);
     if (P.dense && active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
@@ -614,14 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       ptx::tma_store_commit();
       ptx::tma_store_wait_read_all();
     } else if (active && row == 0 && !*reinterpret_cast<volatile int *>(&c.abort)) {
-      const PlanTile &tile = P.plan.tile[ty.first_tile + q_tile0 + g];
-      for (int i = 0; i < tile.n_pieces; ++i) {
-        const PlanPiece pc = P.plan.piece[tile.first_piece + i];
-        const int x = wrap(ox + pc.lx, P.g.W), y = wrap(oy + pc.ly, P.g.H), t = wrap(ot + pc.lt, P.g.T);
-        const uint8_t *src = q_tile + uint32_t(pc.dest) * 128u;
-        ptx::tma_store_5d(&P.map_o[pc.shape], src, 0, x, y, t, bh);
-        ptx::tma_store_5d(&P.map_o[pc.shape], src + kHalfBytes, 64, x, y, t, bh);
-      }
+      const int org[3] = {ot, oy, ox};
+      sm100::store_window_tile(P.plan, P.g, P.map_o, P.plan.tile[ty.first_tile + q_tile0 + g], org, bh, q_tile);
       ptx::tma_store_commit();
       ptx::tma_store_wait_read_all();
     }
@@ -636,34 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encoder(); }
-
-// 5-D map (d, x, y, t, b*head) over the visual rows of a [B, heads, rows, 128] tensor.
-bool encode_grid_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh,
-                     const PlanShape &s) {
-  const cuuint64_t e = 2;
-  cuuint64_t dims[5] = {cuuint64_t(p.head_dim), cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.T),
-                        cuuint64_t(p.B) * cuuint64_t(p.heads)};
-  cuuint64_t strides[4] = {p.head_dim * e, cuuint64_t(p.W) * p.head_dim * e, cuuint64_t(p.H) * p.W * p.head_dim * e,
-                           cuuint64_t(rows_per_bh) * p.head_dim * e};
-  cuuint32_t box[5] = {64, cuuint32_t(s.cx), cuuint32_t(s.cy), cuuint32_t(s.ct), 1};
-  cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3-D map (d, row, b*head) with 128-row boxes; rows past the end read as zero.
-bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh) {
-  const cuuint64_t e = 2;
-  cuuint64_t dims[3] = {cuuint64_t(p.head_dim), cuuint64_t(rows_per_bh), cuuint64_t(p.B) * cuuint64_t(p.heads)};
-  cuuint64_t strides[2] = {p.head_dim * e, cuuint64_t(rows_per_bh) * p.head_dim * e};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 basa_status run_attn(const AttnParams &P, long long blocks, cudaStream_t s) {
   if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
@@ -684,6 +566,46 @@ int text_splits(const basa_params &p, int sms) {
 }
 
 }  // namespace
+
+// 5-D map (d, x, y, t, b*head) over the visual rows of a [B, heads, rows, 128] tensor.
+bool encode_grid_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh,
+                     const PlanShape &s) {
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {cuuint64_t(p.head_dim), cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.T),
+                        cuuint64_t(p.B) * cuuint64_t(p.heads)};
+  cuuint64_t strides[4] = {p.head_dim * e, cuuint64_t(p.W) * p.head_dim * e, cuuint64_t(p.H) * p.W * p.head_dim * e,
+                           cuuint64_t(rows_per_bh) * p.head_dim * e};
+  cuuint32_t box[5] = {64, cuuint32_t(s.cx), cuuint32_t(s.cy), cuuint32_t(s.ct), 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map (d, row, b*head) with 128-row boxes; rows past the end read as zero.
+bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh) {
+  const cuuint64_t e = 2;
+  cuuint64_t dims[3] = {cuuint64_t(p.head_dim), cuuint64_t(rows_per_bh), cuuint64_t(p.B) * cuuint64_t(p.heads)};
+  cuuint64_t strides[2] = {p.head_dim * e, cuuint64_t(rows_per_bh) * p.head_dim * e};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 5-D map (4, x, y, t, b*head) over [B*heads, N, 4] float32 records, no swizzle.
+bool encode_record_map(CUtensorMap *m, const void *base, const basa_params &p, const PlanShape &s) {
+  const cuuint64_t e = 4;
+  const cuuint64_t N = cuuint64_t(p.T) * p.H * p.W;
+  cuuint64_t dims[5] = {4, cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.T), cuuint64_t(p.B) * cuuint64_t(p.heads)};
+  cuuint64_t strides[4] = {4 * e, cuuint64_t(p.W) * 4 * e, cuuint64_t(p.H) * p.W * 4 * e, N * 4 * e};
+  cuuint32_t box[5] = {4, cuuint32_t(s.cx), cuuint32_t(s.cy), cuuint32_t(s.ct), 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<void *>(base), dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -712,7 +634,7 @@ int device_sm_count() {
 basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                              const int32_t *route_idx, void *out, float *lse, uint32_t keys, const basa_params &p,
                              cudaStream_t s) {
-  if (!encode_fn()) return BASA_ERR_CUDA;
+  if (!tensor_map_encoder()) return BASA_ERR_CUDA;
   AttnParams P;
   std::memset(&P, 0, sizeof(P));
   basa_status st = build_window_plan(p, &P.plan);
@@ -763,7 +685,7 @@ size_t text_attn_workspace(const basa_params &p, int sms) {
 
 basa_status launch_attn_text_bf16(const void *q_text, const void *k, const void *v, void *out_text, void *workspace,
                                   const basa_params &p, int sms, cudaStream_t s) {
-  if (!encode_fn()) return BASA_ERR_CUDA;
+  if (!tensor_map_encoder()) return BASA_ERR_CUDA;
   AttnParams P;
   std::memset(&P, 0, sizeof(P));
   P.g = make_geo(p);

@@ -157,6 +157,11 @@ size_t attn_bwd_workspace(const basa_params &p);
 basa_status launch_attn_bwd_f32(const void *q, const void *k, const void *v, const void *kp, const void *vp,
                                 const int32_t *route_idx, const void *out, const float *lse, const void *dout,
                                 void *dq, void *dk, void *dv, void *workspace, const basa_params &p, cudaStream_t s);
+// Backward of the attention, bfloat16 (tensor cores), head_dim 128; deterministic.
+size_t attn_bwd_bf16_workspace(const basa_params &p);
+basa_status launch_attn_bwd_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
+                                 const int32_t *route_idx, const void *out, const float *lse, const void *dout,
+                                 void *dq, void *dk, void *dv, void *workspace, const basa_params &p, cudaStream_t s);
 basa_status launch_attn_text_f32(const void *q_text, const void *k, const void *v, void *out_text,
                                  const basa_params &p, cudaStream_t s);
 

@@ -137,8 +137,9 @@ class BasaLayer:
         B.basa_text_attn_fwd(q_text, k, v, out_text, ws, self.params((0, 0, 0)), stream)
 
     def backward(self, q, k, v, out, lse, dout, shift, stream=None):
-        """dq, dk, dv of the attention (float32; basa_window_attn_bwd) for the pooled
-        K/V and routed windows currently held by the layer."""
+        """dq, dk, dv of the attention (basa_window_attn_bwd: bfloat16 on the tensor
+        cores, or float32) for the pooled K/V and routed windows currently held by
+        the layer; `lse` is the forward's log-sum-exp over all keys."""
         dq = torch.empty_like(q)
         dk = torch.empty_like(k)
         dv = torch.empty_like(v)

@@ -172,8 +172,13 @@ def test_text_attn_checks():
 def test_backward_checks():
     pf = _p(dtype="f32")
     args = [FAKE] * 5 + [None] + [FAKE] * 7
-    assert B.basa_window_attn_bwd(*args, _p(), stream=0, check=False) == 3  # bfloat16: not built
     assert B.basa_window_attn_bwd(*args, _p(dtype="f32", head_dim=64), stream=0, check=False) == 3
+    assert B.basa_window_attn_bwd(*args, _p(head_dim=64), stream=0, check=False) == 3  # bfloat16 needs 128
+    bad = list(args)
+    bad[12] = FAKE + 16  # bfloat16: the workspace must be 256-byte aligned
+    assert B.basa_window_attn_bwd(*bad, _p(), stream=0, check=False) == 1
+    bad[12] = None
+    assert B.basa_window_attn_bwd(*bad, _p(), stream=0, check=False) == 1
     bad = list(args)
     bad[8] = None  # no dout
     assert B.basa_window_attn_bwd(*bad, pf, stream=0, check=False) == 1
