@@ -22,7 +22,8 @@ source), `hbm_kernels` (the pooling / routing pre-pass against measured HBM
 bandwidth), `e2e` (the same metric through BasaLayer.forward with pinned host
 buffers, copies of successive steps pipelined over three streams), `clocks`,
 `cpu_baseline` and context lines for the other workloads and forms (Wan 480p and
-video, the branch form, the text-query rows, the float32 backward).
+video, the branch form, the text-query rows, the bfloat16 tensor-core backward on
+the FLUX 2048^2 and Wan shapes, the float32 backward).
 
 The reference arm (--impl reference) times the float64 CPU oracle on the host
 cores on a bounded sample of the same workload (the oracle is the only other
@@ -369,6 +370,7 @@ def run_ours(args, world, rank, local):
         res["branch_form"] = run_branch_form(args, layer, qd, kd, vd, shifts, flops)
         if wl.n_text > 0:
             res["text_queries"] = run_text_queries(args, layer, wl, kd, vd)
+        res["backward_bf16"] = {n: run_backward_bf16(args, n, synth.SHIFT_CYCLES[n][-1]) for n in ("flux2k", "wan")}
         res["backward_f32"] = run_backward(args)
         for name in ("wan", "wan_video", "flux1k", "flux4k"):
             if args.workload != name:
@@ -437,6 +439,51 @@ def run_backward(args):
     return {"workload": "flux1k shape, float32, shift (0, 8, 8)", "ms": round(ms, 3),
             "gflop": round(flops / 1e9, 2), "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "note": "CUDA-core float32 with atomic dK/dV accumulation; no tensor-core backward yet"}
+
+
+def run_backward_bf16(args, name, shift):
+    """The tensor-core backward (bfloat16) of one layer of workload `name` at `shift`:
+    dq, dk, dv from the forward's output and log-sum-exp. Algorithmic FLOPs = 2.5 x
+    the forward's (the five products S, dP, dq, dK, dV); the kernels execute 3.5 x
+    (the dK/dV pass recomputes S and dP instead of accumulating dq with atomics)."""
+    from sparse_window_attention_b200 import binding as B
+    from sparse_window_attention_b200.layer import BasaLayer
+
+    wl = synth.WORKLOADS[name]
+    q, k, v = synth.make_inputs(wl, seed=args.seed)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    layer = BasaLayer(wl.B, wl.heads, wl.d, wl.grid, wl.window, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
+                      route_radius=wl.route_radius)
+    layer.forward(qd, kd, vd, shift)  # pooled K/V and routes
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=qd.device)
+    layer.attention_lse(qd, kd, vd, out, lse, shift, B.BASA_KEYS_ALL)
+    g = torch.Generator(device="cpu").manual_seed(args.seed + 7)
+    dout = torch.randn(qd.shape, generator=g).to(torch.bfloat16).cuda()
+    for _ in range(3):
+        layer.backward(qd, kd, vd, out, lse, dout, shift)
+    torch.cuda.synchronize()
+    steps = max(10, args.steps // 10)
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        layer.backward(qd, kd, vd, out, lse, dout, shift)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    ms = t0.elapsed_time(t1) / steps
+    cnt = accounting.workload_counts(wl)
+    alg = 2.5 * cnt["attn_flops"]
+    executed = 3.5 * cnt["attn_flops"]
+    peaks, _ = load_peaks()
+    return {"workload": f"{name}, shift {tuple(shift)}, bfloat16", "ms": round(ms, 4),
+            "algorithmic_gflop": round(alg / 1e9, 2), "value": round(alg / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "frac_of_measured_bf16": round(alg / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "executed_tensor_tflops": round(executed / (ms * 1e-3) / 1e12, 2),
+            "executed_frac_of_measured_bf16": round(executed / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "launches_per_step": 5 if (layer.has_pool or layer.n_text) else 3,
+            "note": "records + dq pass + pooled/text dK/dV chunks + chunk reduction + window dK/dV; deterministic"}
 
 
 def run_branch_form(args, layer, qd, kd, vd, shifts, flops):

@@ -175,6 +175,12 @@ __device__ __forceinline__ const PlanTile &q_tile(const BwdParams &P, const QIte
   return P.plan.tile[P.plan.type[it.type].first_tile + it.t];
 }
 
+// dq pass ring: key tile j in slot j % 3 (read by S(j) and, much later, dq(j)),
+// value tile j in slot 3 (read by dP(j) only), so the next key tiles load while
+// earlier ones still wait for their dq product.
+__device__ __forceinline__ int dq_slot(int j, bool is_v) { return is_v ? 3 : j % 3; }
+__device__ __forceinline__ uint32_t dq_phase(int j, bool is_v) { return is_v ? (j & 1) : ((j / 3) & 1); }
+
 // Packs 64 fp32 values (pairs 2i, 2i+1) into 32 bf16x2 words.
 __device__ __forceinline__ void pack64(const float (&x)[64], uint32_t (&w)[32]) {
 #pragma unroll
@@ -336,21 +342,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tma_load_3d(row1, mv, &c.row_full, 0, row, bh);
         ptx::tma_load_3d(row1 + kHalfBytes, mv, &c.row_full, 64, row, bh);
       }
-      int last = -1;
+      int last = -1, last_k = -1, last_v = -1;
       if (MODE == kDq) {
         KeyIter it;
         key_first(P, c, it);
         for (int j = 0; j < n_cols; ++j) {
           bool ok = true;
           for (int kv = 0; kv < 2; ++kv) {
-            const int item = 2 * j + kv, slot = item % kSlots;
-            if (!wt.wait(&c.empty[slot], ((item / kSlots) & 1) ^ 1)) { ok = false; break; }
+            const int slot = dq_slot(j, kv == 1);
+            if (!wt.wait(&c.empty[slot], dq_phase(j, kv == 1) ^ 1)) { ok = false; break; }
             const uint32_t bytes = it.seg <= P.routed_k
                                        ? uint32_t(P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t].valid_rows) * 256u
                                        : kTileBytes;
             ptx::mbar_arrive_expect_tx(&c.full[slot], bytes);
             load_key(P, c, it, kv == 1, bh, smem + kSmemRing + slot * kTileBytes, &c.full[slot]);
-            last = item;
+            (kv ? last_v : last_k) = j;
           }
           if (!ok) break;
           key_next(P, c, it);
@@ -381,7 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         }
       }
       // Drain: wait for the copies still in flight (immediate when all were consumed).
+      // A slot's earlier copies completed before the slot was granted again.
       drain.wait(&c.row_full, 0);
+      if (MODE == kDq) {
+        for (int j = max(0, last_k - 2); j <= last_k; ++j) drain.wait(&c.full[dq_slot(j, false)], dq_phase(j, false));
+        if (last_v >= 0) drain.wait(&c.full[dq_slot(last_v, true)], dq_phase(last_v, true));
+      }
       for (int item = max(0, last - (kSlots - 1)); item <= last; ++item)
         drain.wait(&c.full[item % kSlots], (item / kSlots) & 1);
     }
@@ -399,48 +410,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       if (MODE == kDq && ok && n_cols > 0) {
         // TMEM: S buffers at 0 and 128, dP at 256, dq at 384
         const uint32_t tS[2] = {tmem, tmem + 128}, tDP = tmem + 256, tDQ = tmem + 384;
-        ok = wt.wait(&c.full[0], 0);
+        auto kdesc = [&](int j) { return ringK + uint32_t(dq_slot(j, false)) * kTileDesc; };
+        auto wait_k = [&](int j) { return wt.wait(&c.full[dq_slot(j, false)], dq_phase(j, false)); };
+        auto wait_v = [&](int j) { return wt.wait(&c.full[dq_slot(j, true)], dq_phase(j, true)); };
+        const uint32_t vdesc = ringK + 3u * kTileDesc;
+        ok = wait_k(0);
         if (ok) {
           ptx::tc_fence_after();
-          issue_ss(tS[0], r0, ringK + slot_of(0));  // S(0) = q K0^T
+          issue_ss(tS[0], r0, kdesc(0));  // S(0) = q K0^T
           ptx::mma_commit(&c.s_full[0]);
-          ok = wt.wait(&c.full[1], 0);
+          ok = wait_v(0);
         }
         if (ok) {
           ptx::tc_fence_after();
-          issue_ss(tDP, r1, ringK + slot_of(1));  // dP(0) = dout V0^T
+          issue_ss(tDP, r1, vdesc);  // dP(0) = dout V0^T
           ptx::mma_commit(&c.dp_full);
-          ptx::mma_commit(&c.empty[1]);
+          ptx::mma_commit(&c.empty[3]);
         }
         if (ok && n_cols > 1) {
-          ok = wt.wait(&c.full[2], 0);
+          ok = wait_k(1);
           if (ok) {
             ptx::tc_fence_after();
-            issue_ss(tS[1], r0, ringK + slot_of(2));  // S(1)
+            issue_ss(tS[1], r0, kdesc(1));  // S(1)
             ptx::mma_commit(&c.s_full[1]);
           }
         }
         for (int j = 0; ok && j < n_cols; ++j) {
           if (j >= 1 && j + 1 < n_cols) {
             // S(j+1) into the buffer dq(j-1) has finished reading
-            const int ki = 2 * (j + 1);
-            if (!wt.wait(&c.full[ki % kSlots], (ki / kSlots) & 1)) break;
+            if (!wait_k(j + 1)) break;
             ptx::tc_fence_after();
-            issue_ss(tS[(j + 1) & 1], r0, ringK + slot_of(ki));
+            issue_ss(tS[(j + 1) & 1], r0, kdesc(j + 1));
             ptx::mma_commit(&c.s_full[(j + 1) & 1]);
           }
           if (!wt.wait(&c.ds_full, j & 1)) break;
           ptx::tc_fence_after();
           if (j + 1 < n_cols) {
-            const int vi = 2 * (j + 1) + 1;
-            if (!wt.wait(&c.full[vi % kSlots], (vi / kSlots) & 1)) break;
+            if (!wait_v(j + 1)) break;
             ptx::tc_fence_after();
-            issue_ss(tDP, r1, ringK + slot_of(vi));  // dP(j+1): dP(j) has been read
+            issue_ss(tDP, r1, vdesc);  // dP(j+1): dP(j) has been read
             ptx::mma_commit(&c.dp_full);
-            ptx::mma_commit(&c.empty[vi % kSlots]);
+            ptx::mma_commit(&c.empty[3]);
           }
-          issue_ts_split(tDQ, tS[j & 1], ringMn + slot_of(2 * j), j > 0);  // dq += dS(j) K_j
-          ptx::mma_commit(&c.empty[(2 * j) % kSlots]);
+          issue_ts_split(tDQ, tS[j & 1], ringMn + uint32_t(dq_slot(j, false)) * kTileDesc, j > 0);  // dq += dS(j) K_j
+          ptx::mma_commit(&c.empty[dq_slot(j, false)]);
         }
       } else if (MODE != kDq && ok && n_cols > 0) {
         // TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384
