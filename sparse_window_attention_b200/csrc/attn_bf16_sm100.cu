@@ -11,7 +11,8 @@
 //               include the cyclic shift (mod the grid), so no rolled copy exists.
 //   warp 1      tcgen05 issuer (one thread): S_g = Q_g K^T and O_g += P_g V with
 //               fp32 accumulators in TMEM (S0, S1, O0, O1: 4 x 128 columns).
-//   warps 2-9   two softmax warpgroups, one per query tile; a thread owns one
+//   warps 2-3   idle (they keep the three warpgroups aligned to the SM sub-partitions)
+//   warps 4-11  two softmax warpgroups, one per query tile; a thread owns one
 //               query row: reads its S row from TMEM, runs the online softmax in
 //               fp32 (base-2 exponent, scale folded in), writes P (bf16) back to
 //               TMEM over its S row (A operand of P V), rescales its O row in TMEM when the running max grows,
@@ -46,7 +47,11 @@ using sm100::kTileDesc;
 using sm100::Waiter;
 using sm100::wrap;
 
-constexpr int kThreads = 320;  // 10 warps
+// 12 warps = three warpgroups: warp 0 loads, warp 1 issues MMAs (warps 2-3 idle),
+// warps 4-7 and 8-11 run the softmax of query tile 0 and 1. Each SM sub-partition
+// then holds one warp of each group (with 10 warps, two sub-partitions held two
+// softmax warps and the register limit forced spills).
+constexpr int kThreads = 384;
 constexpr int kStages = 5;
 constexpr uint32_t kSmemQ = 0;                         // 2 query tiles (reused for the output)
 constexpr uint32_t kSmemRing = 2 * kTileBytes;         // K/V ring
@@ -392,10 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
       drain.wait(&c.drain, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
     // Two warpgroups, one per query tile; a thread owns one query row.
-    const int g = (warp - 2) / 4;
+    const int g = (warp - 4) / 4;
     const int sub = warp % 4;  // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;
     const uint32_t lane_off = uint32_t(sub * 32) << 16;
@@ -408,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     {
       // Column masks of this CTA's key tiles in stream order (all ones = full tile),
       // one tile per softmax thread; this runs while the first loads are in flight.
-      const int j = threadIdx.x - 64;
+      const int j = threadIdx.x - 128;
       if (j < kMaskTable && j < n_kt) {
         KeyIter t{0, j};
         while (t.seg <= P.routed_k + 2 && t.t >= seg_tiles(P, c, t.seg)) {
