@@ -735,6 +735,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="flux2k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--part", default="layer", choices=["layer", "backward"],
+                    help="layer: the forward layer (the metric); backward: only the bfloat16 backward of the "
+                         "workload at the last shift of its cycle (a context figure, e.g. for profiling)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="replicas: a full layer per GPU (weak scaling); heads: one layer's (batch, head) units "
                          "split over the GPUs (strong scaling)")
@@ -756,6 +759,11 @@ def main():
         return
 
     world, rank, local = dist_setup()
+    if args.part == "backward":
+        if rank == 0:
+            print(json.dumps({"backward_bf16": run_backward_bf16(args, args.workload,
+                                                                 synth.SHIFT_CYCLES[args.workload][-1])}), flush=True)
+        return
     res = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(args)
