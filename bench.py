@@ -79,11 +79,28 @@ def kernel_traffic(kernel_file: str, workload: str):
     return float(m_tr.group(1))
 
 
+_NVML_POLL = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+bus = sys.argv[1]
+h = pynvml.nvmlDeviceGetHandleByPciBusId(bus) if bus else pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    t = time.time()
+    print(f"{t:.6f} {pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)} "
+          f"{int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))}", flush=True)
+    time.sleep(0.0005)
+"""
+
+
 class ClockSampler:
     """SM clocks and throttle reasons sampled DURING the timed region.
 
-    NVML is polled from a thread every ~0.5 ms (a timed region of a few ms still
-    gets samples); without NVML, `nvidia-smi -lms 100` is the fallback."""
+    A separate process polls NVML every ~0.5 ms (no GIL contention with the
+    launching thread) and timestamps each sample; the samples inside the timed
+    region's wall-clock interval are kept, so a region of a few ms still gets a
+    handful. Without NVML, `nvidia-smi -lms 100` is the fallback."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))
@@ -92,75 +109,76 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.stop = threading.Event()
-        self.samples = []  # (sm_mhz, reason bits)
-        self.max_mhz = None
         self.lines = []
+        self.max_mhz = None
         self.source = None
-
-    def _nvml_handle(self):
-        import pynvml
-
-        pynvml.nvmlInit()
-        try:  # the device torch uses, whatever CUDA_VISIBLE_DEVICES says
-            pr = torch.cuda.get_device_properties(self.index)
-            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-        except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
+        bus = ""
         try:
-            nv, h = self._nvml_handle()
-            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
-            self.source = "nvml, every 0.5 ms"
-
-            def poll():
-                while not self.stop.is_set():
-                    try:
-                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
-                                             int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
-                    except Exception:
-                        break
-                    time.sleep(0.0005)
-
-            self.thread = threading.Thread(target=poll, daemon=True)
-            self.thread.start()
-            return self
+            pr = torch.cuda.get_device_properties(self.index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
         except Exception:
             pass
         try:
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLL, bus, str(self.index)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            first = self.proc.stdout.readline().split()
+            if len(first) != 2 or first[0] != "max":
+                raise OSError("nvml poller did not start")
+            self.max_mhz = float(first[1])
+            self.source = "nvml from a separate process, every 0.5 ms"
+        except Exception:
+            if self.proc is not None:
+                self.proc.kill()
             self.source = "nvidia-smi -lms 100"
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100", "-i", str(self.index)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100", "-i",
+                     str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (FileNotFoundError, OSError):
+                self.proc = None
+                self.source = None
+        if self.proc is not None:
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-        except (FileNotFoundError, OSError):
-            self.proc = None
-            self.source = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *a):
-        self.stop.set()
         if self.proc is not None:
+            time.sleep(0.002)  # let the poller report past the end of the region
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-        if getattr(self, "thread", None) is not None:
             self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [s for s, _ in self.samples], self.max_mhz, set()
-        for _, bits in self.samples:
-            reasons.update(n for n, b in self.REASONS if bits & b)
+        sm, mx, reasons = [], self.max_mhz, set()
+        nvml = self.source is not None and self.source.startswith("nvml")
         for line in self.lines:
+            if nvml:
+                parts = line.split()
+                if len(parts) != 3:
+                    continue
+                t, mhz, bits = float(parts[0]), float(parts[1]), int(parts[2])
+                if self.t0 is not None and not (self.t0 <= t <= self.t1):
+                    continue
+                sm.append(mhz)
+                reasons.update(n for n, b in self.REASONS if bits & b)
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
@@ -172,9 +190,8 @@ class ClockSampler:
             for (n, _), v in zip(self.REASONS, parts[3:7]):
                 if v.lower() == "active":
                     reasons.add(n)
-        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-               "samples": len(sm), "source": self.source}
-        return out
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "source": self.source}
 
 
 def dist_setup():
@@ -262,11 +279,13 @@ def run_ours(args, world, rank, local):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     with sampler:
+        sampler.mark_start()
         t0.record(stream)
         for i in range(args.steps):
             step(i)
         t1.record(stream)
         torch.cuda.synchronize()
+        sampler.mark_end()
     barrier(world)
     step_ms = t0.elapsed_time(t1) / args.steps
     step_ms = max_over_ranks(step_ms, world)
@@ -438,7 +457,8 @@ def run_backward(args):
     flops = 2.5 * cnt["attn_flops"]
     return {"workload": "flux1k shape, float32, shift (0, 8, 8)", "ms": round(ms, 3),
             "gflop": round(flops / 1e9, 2), "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "note": "CUDA-core float32 with atomic dK/dV accumulation; no tensor-core backward yet"}
+            "note": "CUDA-core float32 with atomic dK/dV accumulation (the bfloat16 backward runs on the tensor cores: "
+                    "backward_bf16)"}
 
 
 def run_backward_bf16(args, name, shift):

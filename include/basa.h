@@ -18,7 +18,7 @@
  *   basa_window_attn_fwd_lse  one branch of the decomposed form, with log-sum-exp
  *   basa_merge_branches       branches merged into the joint softmax  (BASA §A.1)
  *   basa_text_attn_fwd        the text queries' output rows (dense over all keys)
- *   basa_window_attn_bwd      gradients w.r.t. q, k, v (float32)       (BASA §3.4)
+ *   basa_window_attn_bwd      gradients w.r.t. q, k, v                 (BASA §3.4)
  *
  * Conventions common to every entry point
  * ---------------------------------------
@@ -250,11 +250,20 @@ basa_status basa_text_attn_fwd(const void *q_text, const void *k, const void *v,
  * the key rows of dK, dV added back to the tokens they came from: own and routed
  * window tokens, text rows, and pooled keys spread evenly over their patch's
  * tokens (kp, vp are means). Routing is a selection and passes no gradient.
- * Outputs (overwritten): dq [B, heads, N, d], dk, dv [B, heads, N + n_text, d].
- * Float32 only, head_dim 128 (BASA_ERR_UNSUPPORTED otherwise). `workspace`
- * (device, 16-byte aligned) holds basa_window_attn_bwd_workspace_bytes(p) bytes
- * for the pooled keys' gradients (NULL when that is 0). dk, dv are accumulated
- * with atomic adds, so their last bits can differ between runs; dq cannot.
+ * Outputs (overwritten): dq [B, heads, N, d], dk, dv [B, heads, N + n_text, d],
+ * element type p->dtype. head_dim 128 only (BASA_ERR_UNSUPPORTED otherwise).
+ * `workspace` is a device buffer of basa_window_attn_bwd_workspace_bytes(p) bytes
+ * (contents on entry ignored):
+ *  - BASA_BF16: tensor cores (tcgen05), 256-byte aligned workspace holding a
+ *    16-byte record {lse log2(e), dout . out} per query token, per-chunk partial
+ *    gradients of the pooled and text keys and the pooled keys' gradients. Every
+ *    sum has a fixed order and nothing is accumulated atomically: the results are
+ *    identical run to run. P and dS are rounded to bfloat16 before the tensor-core
+ *    products, each output once at the end. With routing, nWin <= 4096.
+ *    BASA_ERR_UNSUPPORTED when the window tiling exceeds the kernel's limits.
+ *  - BASA_F32: CUDA cores, 16-byte aligned workspace for the pooled keys'
+ *    gradients (NULL when that is 0); dk, dv are accumulated with atomic adds, so
+ *    their last bits can differ between runs; dq cannot.
  */
 size_t basa_window_attn_bwd_workspace_bytes(const basa_params *p);
 basa_status basa_window_attn_bwd(const void *q, const void *k, const void *v,
