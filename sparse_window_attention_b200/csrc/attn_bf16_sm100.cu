@@ -69,12 +69,21 @@ struct alignas(64) AttnParams {
   CUtensorMap map_v[kMaxShapes];
   CUtensorMap map_o[kMaxShapes];
   CUtensorMap map_kp, map_vp, map_kt, map_vt;
+  CUtensorMap map_kp8, map_vp8;  // pooled rows in 8-row boxes (the pooled tail, see below)
   CUtensorMap map_qd, map_od;  // text-query mode: query rows and output rows (d, row, b*head)
   WindowPlan plan;
   const int32_t *route;
   int32_t *dev_err;
   Geo g;
   int routed_k, n_pool, n_text, n_pool_tiles, n_text_tiles;
+  // Pooled tail: when the pooled keys past the last full 128-row tile (pool_tail rows,
+  // at most 16) fit in free 8-row blocks of the own window's key tile tail_tile[type],
+  // they are loaded there (8-row boxes at rows tail_dest[type][b]) instead of taking a
+  // key tile of their own; tail_mask[type] marks their rows.
+  int pool_tail, tail_blocks;
+  int8_t tail_tile[8];
+  uint8_t tail_dest[8][2];
+  uint32_t tail_mask[8][4];
   float scale_log2;
   int use_windows;  // own and routed windows are keys (else pooled and/or text only)
   // Text-query mode: the queries are the n_text text rows and attend densely to
@@ -128,11 +137,35 @@ __device__ __forceinline__ KeyIter first_key(const AttnParams &P, const Ctrl &c)
   return it;
 }
 
+// The own window's key tile that also carries the pooled tail.
+__device__ __forceinline__ bool has_pool_tail(const AttnParams &P, const Ctrl &c, const KeyIter &it) {
+  return P.pool_tail > 0 && it.seg == 0 && it.t == P.tail_tile[c.wtype[0]];
+}
+
+// Bytes the TMA loads of one key (or value) tile deliver.
+__device__ __forceinline__ uint32_t key_tile_bytes(const AttnParams &P, const Ctrl &c, const KeyIter &it) {
+  if (it.seg > P.routed_k) return kTileBytes;  // whole 128-row boxes (rows past the end read as zero)
+  uint32_t b = uint32_t(P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t].valid_rows) * 256u;
+  if (has_pool_tail(P, c, it)) b += uint32_t(P.tail_blocks) * 8u * 256u;
+  return b;
+}
+
 __device__ __forceinline__ uint32_t load_key_tile(const AttnParams &P, const Ctrl &c, const KeyIter &it, bool is_v,
                                                   int bh, uint8_t *dst, uint64_t *bar) {
   if (it.seg <= P.routed_k) {
     const PlanTile &tile = P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t];
-    return sm100::load_window_tile(P.plan, P.g, is_v ? P.map_v : P.map_k, tile, c.org[it.seg], bh, dst, bar);
+    uint32_t b = sm100::load_window_tile(P.plan, P.g, is_v ? P.map_v : P.map_k, tile, c.org[it.seg], bh, dst, bar);
+    if (has_pool_tail(P, c, it)) {
+      const CUtensorMap *map = is_v ? &P.map_vp8 : &P.map_kp8;
+      for (int i = 0; i < P.tail_blocks; ++i) {
+        uint8_t *d = dst + uint32_t(P.tail_dest[c.wtype[0]][i]) * 128u;
+        const int row = P.n_pool_tiles * kTileRows + 8 * i;  // rows past n_pool read as zero
+        ptx::tma_load_3d(d, map, bar, 0, row, bh);
+        ptx::tma_load_3d(d + kHalfBytes, map, bar, 64, row, bh);
+        b += 8u * 256u;
+      }
+    }
+    return b;
   }
   const bool pooled = it.seg == P.routed_k + 1;
   const CUtensorMap *map = pooled ? (is_v ? &P.map_vp : &P.map_kp) : (is_v ? &P.map_vt : &P.map_kt);
@@ -148,6 +181,11 @@ __device__ __forceinline__ bool key_tile_mask(const AttnParams &P, const Ctrl &c
     const PlanTile &tile = P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t];
 #pragma unroll
     for (int i = 0; i < 4; ++i) m[i] = tile.mask[i];
+    if (has_pool_tail(P, c, it)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[i] |= P.tail_mask[c.wtype[0]][i];
+      return false;
+    }
     return tile.valid_rows == kTileRows;
   }
   const bool pooled = it.seg == P.routed_k + 1;
@@ -322,9 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
           if (item == 0 && (P.flags & BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD)) { skipped0 = true; last = item; continue; }
           uint8_t *dst = smem + kSmemRing + slot * kTileBytes;
           // Arm the barrier with the byte count before issuing the copies.
-          const uint32_t bytes = it.seg <= P.routed_k
-                                     ? uint32_t(P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t].valid_rows) * 256u
-                                     : kTileBytes;
+          const uint32_t bytes = key_tile_bytes(P, c, it);
           ptx::mbar_arrive_expect_tx(&c.full[slot], bytes);
           load_key_tile(P, c, it, kv == 1, bh, dst, &c.full[slot]);
           last = item;
@@ -552,6 +588,48 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
 
 // ----------------------------------------------------------------- host side
 
+// Pooled tail: the pooled keys past the last full tile (1..16 rows) go into free
+// 8-row blocks of one key tile of the own window when every window type has such
+// blocks; the pooled segment then has one tile fewer. Returns whether it is on.
+bool plan_pool_tail(AttnParams &P) {
+  const int tail = P.n_pool % kTileRows;
+  if (tail == 0 || tail > 16) return false;
+  const int blocks = (tail + 7) / 8;
+  int8_t tile_of[8];
+  uint8_t dest[8][2];
+  uint32_t mask[8][4];
+  for (int ty = 0; ty < 8; ++ty) {
+    tile_of[ty] = -1;
+    const PlanType &pt = P.plan.type[ty];
+    // a type no window has keeps tile -1 (never matched)
+    for (int t = pt.n_tiles - 1; t >= 0 && tile_of[ty] < 0; --t) {
+      const PlanTile &tile = P.plan.tile[pt.first_tile + t];
+      int found = 0;
+      for (int b = 0; b < kTileRows / 8 && found < blocks; ++b) {
+        bool free_block = true;
+        for (int r = 8 * b; r < 8 * b + 8; ++r) free_block &= !((tile.mask[r >> 5] >> (r & 31)) & 1u);
+        if (free_block) dest[ty][found++] = uint8_t(8 * b);
+      }
+      if (found == blocks) tile_of[ty] = int8_t(t);
+    }
+    if (pt.n_tiles > 0 && tile_of[ty] < 0) return false;
+    for (int i = 0; i < 4; ++i) mask[ty][i] = 0;
+    if (tile_of[ty] >= 0)
+      for (int b = 0; b < blocks; ++b)
+        for (int r = 0; r < 8 && 8 * b + r < tail; ++r) {
+          const int row = dest[ty][b] + r;
+          mask[ty][row >> 5] |= 1u << (row & 31);
+        }
+  }
+  P.pool_tail = tail;
+  P.tail_blocks = blocks;
+  P.n_pool_tiles = P.n_pool / kTileRows;
+  std::memcpy(P.tail_tile, tile_of, sizeof(tile_of));
+  std::memcpy(P.tail_dest, dest, sizeof(dest));
+  std::memcpy(P.tail_mask, mask, sizeof(mask));
+  return true;
+}
+
 basa_status run_attn(const AttnParams &P, long long blocks, cudaStream_t s) {
   if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return BASA_ERR_CUDA;
@@ -587,12 +665,12 @@ bool encode_grid_map(CUtensorMap *m, const void *base, const basa_params &p, lon
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map (d, row, b*head) with 128-row boxes; rows past the end read as zero.
-bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh) {
+// 3-D map (d, row, b*head) with box_rows-row boxes; rows past the end read as zero.
+bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh, int box_rows) {
   const cuuint64_t e = 2;
   cuuint64_t dims[3] = {cuuint64_t(p.head_dim), cuuint64_t(rows_per_bh), cuuint64_t(p.B) * cuuint64_t(p.heads)};
   cuuint64_t strides[2] = {p.head_dim * e, cuuint64_t(rows_per_bh) * p.head_dim * e};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -664,6 +742,10 @@ basa_status launch_attn_bf16(const void *q, const void *k, const void *v, const 
     if (!encode_rows_map(&P.map_kt, k, p, kv_rows) || !encode_rows_map(&P.map_vt, v, p, kv_rows)) return BASA_ERR_CUDA;
   }
   P.n_pool_tiles = (keys & BASA_KEYS_POOLED) ? (P.n_pool + kTileRows - 1) / kTileRows : 0;
+  if ((keys & BASA_KEYS_POOLED) && (keys & BASA_KEYS_WINDOWS) && plan_pool_tail(P)) {
+    if (!encode_rows_map(&P.map_kp8, kp, p, P.n_pool, 8) || !encode_rows_map(&P.map_vp8, vp, p, P.n_pool, 8))
+      return BASA_ERR_CUDA;
+  }
   P.n_text_tiles = (keys & BASA_KEYS_TEXT) ? (p.n_text + kTileRows - 1) / kTileRows : 0;
   P.use_windows = (keys & BASA_KEYS_WINDOWS) ? 1 : 0;
   P.lse = lse;

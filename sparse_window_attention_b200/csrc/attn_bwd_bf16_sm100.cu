@@ -750,7 +750,12 @@ int head_query_tiles(const basa_params &p, const WindowPlan &plan) {
   return n;
 }
 
-BwdLayout bwd_layout(const basa_params &p, const WindowPlan &plan, int sms) {
+// Chunking of the pooled / text key tiles' query range: enough CTAs for about two
+// waves of a 148-SM part, at least 4 query tiles per chunk. It depends on the shape
+// only, so the workspace size and the order of the chunk sums (hence the bits of the
+// results) are the same on every device.
+constexpr long long kLongTargetCtas = 2 * 148;
+BwdLayout bwd_layout(const basa_params &p, const WindowPlan &plan) {
   BwdLayout L{};
   const long long bh = (long long)p.B * p.heads;
   const long long N = (long long)p.T * p.H * p.W;
@@ -759,9 +764,8 @@ BwdLayout bwd_layout(const basa_params &p, const WindowPlan &plan, int sms) {
   L.q_tiles = head_query_tiles(p, plan);
   L.n_chunks = 1;
   if (L.n_long > 0) {
-    // enough CTAs for two waves, at least 4 query tiles per chunk
     const long long units = bh * L.n_long;
-    long long want = (2LL * std::max(sms, 1) + units - 1) / units;
+    long long want = (kLongTargetCtas + units - 1) / units;
     want = std::max(1LL, std::min<long long>(want, std::max(1, L.q_tiles / 4)));
     L.chunk_tiles = int((L.q_tiles + want - 1) / want);
     L.n_chunks = (L.q_tiles + L.chunk_tiles - 1) / L.chunk_tiles;
@@ -789,7 +793,7 @@ basa_status run_bwd(const BwdParams &P, long long blocks, cudaStream_t s) {
 size_t attn_bwd_bf16_workspace(const basa_params &p) {
   static thread_local WindowPlan plan;  // large: kept off the stack
   if (build_window_plan(p, &plan) != BASA_OK) return 0;
-  return bwd_layout(p, plan, device_sm_count()).total;
+  return bwd_layout(p, plan).total;
 }
 
 basa_status launch_attn_bwd_bf16(const void *q, const void *k, const void *v, const void *kp, const void *vp,
@@ -800,9 +804,7 @@ basa_status launch_attn_bwd_bf16(const void *q, const void *k, const void *v, co
   std::memset(&P, 0, sizeof(P));
   basa_status st = build_window_plan(p, &P.plan);
   if (st != BASA_OK) return st;
-  const int sms = device_sm_count();
-  if (sms <= 0) return BASA_ERR_CUDA;
-  const BwdLayout L = bwd_layout(p, P.plan, sms);
+  const BwdLayout L = bwd_layout(p, P.plan);
   P.g = make_geo(p);
   if (p.routed_k > 0 && P.g.nWin > kMaxList) return BASA_ERR_UNSUPPORTED;
   const long long N = P.g.N, kv_rows = N + p.n_text, bh = (long long)p.B * p.heads;

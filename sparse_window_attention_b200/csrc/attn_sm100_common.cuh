@@ -187,9 +187,11 @@ __device__ __forceinline__ void prefix_mask(int valid, uint32_t *m) {
 // tensor, box = one plan shape, 128-byte swizzle.
 bool encode_grid_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh,
                      const PlanShape &s);
-// 3-D map (d, row, b*head) over a [B*heads, rows, 128] bf16 tensor with 128-row
-// boxes, 128-byte swizzle; rows past the end read as zero and are not stored.
-bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh);
+// 3-D map (d, row, b*head) over a [B*heads, rows, 128] bf16 tensor with box_rows-row
+// boxes (128 unless given), 128-byte swizzle; rows past the end read as zero and are
+// not stored.
+bool encode_rows_map(CUtensorMap *m, const void *base, const basa_params &p, long long rows_per_bh,
+                     int box_rows = 128);
 // 5-D map (4, x, y, t, b*head) over a [B*heads, N, 4] float32 per-token record
 // array, box = one plan shape, no swizzle (16-byte records).
 bool encode_record_map(CUtensorMap *m, const void *base, const basa_params &p, const PlanShape &s);

@@ -187,6 +187,12 @@ def test_backward_checks():
     assert B.basa_window_attn_bwd(*bad, pf, stream=0, check=False) == 1
     # pooled gradients: 2 x heads x 64 patches x 128 floats
     assert B.basa_window_attn_bwd_workspace_bytes(pf) == 2 * 2 * 64 * 128 * 4
+    # bfloat16 (computed on the host, the same on every device): per-token records
+    # (2 heads x 4096 tokens x 16 B), chunk partials of the pooled and text key tiles
+    # (2 heads x 2 tiles x 8 chunks of the 32 query tiles x [dK | dV] x 128 x 128 floats),
+    # pooled-key gradients (2 x 2 heads x 64 x 128 floats)
+    rec, part, pooled = 2 * 4096 * 16, 2 * 2 * 8 * 2 * 128 * 128 * 4, 2 * 2 * 64 * 128 * 4
+    assert B.basa_window_attn_bwd_workspace_bytes(_p()) == rec + part + pooled
 
 
 def test_route_workspace_bytes():
