@@ -68,7 +68,8 @@ typedef enum {
   BASA_ERR_SHAPE = 2,          /* window or pool patch does not divide the grid, shift out of range */
   BASA_ERR_UNSUPPORTED = 3,    /* valid but not built: e.g. bfloat16 attention with head_dim 64 */
   BASA_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
-  BASA_ERR_DEVICE_TIMEOUT = 5  /* a bounded wait inside a kernel expired (reported via dev_err) */
+  BASA_ERR_DEVICE_TIMEOUT = 5, /* a bounded wait inside a kernel expired (reported via dev_err) */
+  BASA_ERR_BAD_INDEX = 6       /* a kernel met an out-of-range route id (reported via dev_err) */
 } basa_status;
 
 typedef enum { BASA_BF16 = 0, BASA_F32 = 1 } basa_dtype;
@@ -77,6 +78,10 @@ typedef enum { BASA_BF16 = 0, BASA_F32 = 1 } basa_dtype;
 #define BASA_DEVERR_TIMEOUT_PRODUCER 0x1
 #define BASA_DEVERR_TIMEOUT_MMA 0x2
 #define BASA_DEVERR_TIMEOUT_SOFTMAX 0x4
+/* A route id outside [0, nWin): the attention kernels (forward and backward) read
+ * the routed window's tokens from the query's own window instead, so nothing is
+ * accessed out of bounds, and set this bit; the results are then not valid. */
+#define BASA_DEVERR_BAD_ROUTE 0x8
 
 /* Test hook for basa_params.flags: the attention kernel's loader skips the TMA
  * load of the first key tile, so every wait on it runs into its time limit and
@@ -191,7 +196,8 @@ basa_status basa_pool_route(const void *q, const void *k, const void *v,
  * accumulators are float32; with BASA_BF16 the products run on the tensor
  * cores in bfloat16 and the output is rounded once to bfloat16.
  * kp, vp must be NULL iff the pool patch is all zero; route_idx must be NULL
- * iff routed_k == 0. Route ids must lie in [0, nWin) (not checked on device).
+ * iff routed_k == 0. Route ids must lie in [0, nWin); the kernel checks them and
+ * reports one outside (BASA_DEVERR_BAD_ROUTE in *dev_err, see there).
  * bfloat16 requires head_dim == 128; float32 supports 64 and 128.
  */
 basa_status basa_window_attn_fwd(const void *q, const void *k, const void *v,
@@ -323,7 +329,8 @@ basa_status basa_route_windows_noalloc(const void *q, const void *k, int32_t *ro
 const char *basa_status_string(basa_status s);
 
 /* Map a device error word (read back from basa_params.dev_err) to a status:
- * 0 -> BASA_OK, any BASA_DEVERR_TIMEOUT_* bit -> BASA_ERR_DEVICE_TIMEOUT. */
+ * 0 -> BASA_OK, BASA_DEVERR_BAD_ROUTE -> BASA_ERR_BAD_INDEX, else (a
+ * BASA_DEVERR_TIMEOUT_* bit) -> BASA_ERR_DEVICE_TIMEOUT. */
 basa_status basa_device_error_status(int32_t dev_err_word);
 
 #ifdef __cplusplus

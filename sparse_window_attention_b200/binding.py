@@ -21,10 +21,12 @@ STATUS_NAMES = {
     3: "BASA_ERR_UNSUPPORTED",
     4: "BASA_ERR_CUDA",
     5: "BASA_ERR_DEVICE_TIMEOUT",
+    6: "BASA_ERR_BAD_INDEX",
 }
 BASA_BF16 = 0
 BASA_F32 = 1
 BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD = 0x1
+BASA_DEVERR_BAD_ROUTE = 0x8
 BASA_KEYS_WINDOWS, BASA_KEYS_POOLED, BASA_KEYS_TEXT, BASA_KEYS_ALL = 1, 2, 4, 7
 BASA_MAX_BRANCHES = 4
 EXPORTED = (

@@ -65,12 +65,14 @@ const char *basa_status_string(basa_status s) {
     case BASA_ERR_UNSUPPORTED: return "BASA_ERR_UNSUPPORTED";
     case BASA_ERR_CUDA: return "BASA_ERR_CUDA";
     case BASA_ERR_DEVICE_TIMEOUT: return "BASA_ERR_DEVICE_TIMEOUT";
+    case BASA_ERR_BAD_INDEX: return "BASA_ERR_BAD_INDEX";
   }
   return "BASA_ERR_UNKNOWN";
 }
 
 basa_status basa_device_error_status(int32_t w) {
-  return w == 0 ? BASA_OK : BASA_ERR_DEVICE_TIMEOUT;
+  if (w == 0) return BASA_OK;
+  return (w & BASA_DEVERR_BAD_ROUTE) ? BASA_ERR_BAD_INDEX : BASA_ERR_DEVICE_TIMEOUT;
 }
 
 basa_status basa_pool_kv(const void *k, const void *v, void *kp, void *vp, const basa_params *p,

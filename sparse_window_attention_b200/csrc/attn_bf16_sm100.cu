@@ -297,7 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bf16_kernel(const __grid_con
     c.wtype[0] = wtype;
     c.org[0][0] = ot; c.org[0][1] = oy; c.org[0][2] = ox;
     for (int r = 0; r < P.routed_k; ++r) {
-      const int u = P.route[((long long)bh * P.g.nWin + w) * P.routed_k + r];
+      int u = P.route[((long long)bh * P.g.nWin + w) * P.routed_k + r];
+      if (u < 0 || u >= P.g.nWin) {  // reported, and replaced by the own window: accesses stay in bounds
+        if (P.dev_err) atomicOr(P.dev_err, BASA_DEVERR_BAD_ROUTE);
+        u = w;
+      }
       int a, b, d, t;
       window_origin(P.g, u, &a, &b, &d, &t);
       c.wtype[1 + r] = t;

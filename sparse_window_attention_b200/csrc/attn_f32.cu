@@ -16,6 +16,7 @@ constexpr int kKeyTile = 32;
 struct F32Args {
   const float *q, *k, *v, *kp, *vp;
   const int32_t *route;
+  int32_t *dev_err;  // nullable: BASA_DEVERR_BAD_ROUTE on an out-of-range route id
   float *out;
   float *lse;  // nullable [B*heads][N]
   Geo g;
@@ -24,6 +25,14 @@ struct F32Args {
   int dense;  // text-query rows: queries are q_text rows, keys are all N + n_text rows of k, v
   float scale;
 };
+
+// A route id outside [0, nWin) is reported (BASA_DEVERR_BAD_ROUTE) and replaced by
+// the query's own window, so every access stays inside the tensors.
+__device__ __forceinline__ int checked_route(const F32Args &a, int u, int w) {
+  if (u >= 0 && u < a.g.nWin) return u;
+  if (a.dev_err) atomicOr(a.dev_err, BASA_DEVERR_BAD_ROUTE);
+  return w;
+}
 
 // Row of key j of window w's key list: [own | routed windows | pooled | text],
 // restricted to the selected groups.
@@ -61,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(F32Args a) {
   const long long bh = blockIdx.x / (a.q_chunks * n_win);
   if (threadIdx.x == 0) wins[0] = w;
   if (!a.dense && threadIdx.x > 0 && threadIdx.x <= a.routed_k)
-    wins[threadIdx.x] = a.route[(bh * a.g.nWin + w) * a.routed_k + threadIdx.x - 1];
+    wins[threadIdx.x] = checked_route(a, a.route[(bh * a.g.nWin + w) * a.routed_k + threadIdx.x - 1], w);
   __syncthreads();
 
   const int half = threadIdx.x % TPQ;
@@ -146,6 +155,7 @@ basa_status launch_attn_f32(const void *q, const void *k, const void *v, const v
   a.kp = static_cast<const float *>(kp);
   a.vp = static_cast<const float *>(vp);
   a.route = route_idx;
+  a.dev_err = p.dev_err;
   a.out = static_cast<float *>(out);
   a.g = make_geo(p);
   a.heads = p.heads;
@@ -244,7 +254,7 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_f32_kernel(BwdArgs b) {
   const long long bh = blockIdx.x / (a.q_chunks * a.g.nWin);
   if (threadIdx.x == 0) wins[0] = w;
   if (threadIdx.x > 0 && threadIdx.x <= a.routed_k)
-    wins[threadIdx.x] = a.route[(bh * a.g.nWin + w) * a.routed_k + threadIdx.x - 1];
+    wins[threadIdx.x] = checked_route(a, a.route[(bh * a.g.nWin + w) * a.routed_k + threadIdx.x - 1], w);
   __syncthreads();
   const int part = threadIdx.x % kBwdTPQ;  // columns part, part + TPQ, ...
   const int lq = chunk * QPB + threadIdx.x / kBwdTPQ;
@@ -375,6 +385,7 @@ basa_status launch_attn_bwd_f32(const void *q, const void *k, const void *v, con
   a.kp = static_cast<const float *>(kp);
   a.vp = static_cast<const float *>(vp);
   a.route = route_idx;
+  a.dev_err = p.dev_err;
   a.g = make_geo(p);
   a.heads = p.heads;
   a.d = p.head_dim;

@@ -30,6 +30,8 @@ def test_status_strings():
         assert B.basa_status_string(code) == name
     assert B.basa_device_error_status(0) == B.BASA_OK
     assert B.basa_device_error_status(2) == 5
+    assert B.basa_device_error_status(B.BASA_DEVERR_BAD_ROUTE) == 6
+    assert B.basa_device_error_status(B.BASA_DEVERR_BAD_ROUTE | 1) == 6
 
 
 def test_params_struct_layout_matches_header():
