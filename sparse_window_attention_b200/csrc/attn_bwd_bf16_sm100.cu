@@ -11,8 +11,8 @@
 //
 // Every sum has a fixed order and nothing is accumulated with atomics, so the
 // results are identical run to run. Launches, in order:
-//   records      per query token {L log2(e), D} (16-byte records, TMA-loadable with
-//                the same boxes as the query tiles)
+//   records      per query token {-L log2(e), -D} (16-byte records, TMA-loadable with
+//                the same boxes as the query tiles; negated for the packed FMA/add)
 //   dq pass      one CTA per (b*head, window, query tile): the key stream of the
 //                forward; S = q K^T and dP = dout V^T on tcgen05 (two S buffers in
 //                TMEM), dS by the compute warps, dq += dS K accumulated in TMEM.
@@ -64,7 +64,7 @@ constexpr uint32_t kTmemCols = 512;
 
 struct alignas(64) BwdParams {
   CUtensorMap map_q[kMaxShapes], map_k[kMaxShapes], map_v[kMaxShapes], map_do[kMaxShapes];
-  CUtensorMap map_rec[kMaxShapes];                 // per-token records {L log2 e, D, 0, 0}
+  CUtensorMap map_rec[kMaxShapes];                 // per-token records {-L log2 e, -D, 0, 0}
   CUtensorMap map_dq[kMaxShapes], map_dk[kMaxShapes], map_dv[kMaxShapes];
   CUtensorMap map_kp, map_vp, map_kt, map_vt;      // pooled and text rows, 128-row boxes
   WindowPlan plan;
@@ -180,6 +180,13 @@ __device__ __forceinline__ const PlanTile &q_tile(const BwdParams &P, const QIte
 // earlier ones still wait for their dq product.
 __device__ __forceinline__ int dq_slot(int j, bool is_v) { return is_v ? 3 : j % 3; }
 __device__ __forceinline__ uint32_t dq_phase(int j, bool is_v) { return is_v ? (j & 1) : ((j / 3) & 1); }
+
+// Sets the columns whose mask bit is clear to 0 (m0: columns 0-31, m1: 32-63).
+__device__ __forceinline__ void zero_masked(float (&x)[64], uint32_t m0, uint32_t m1) {
+#pragma unroll
+  for (int i = 0; i < 64; ++i)
+    if (!(((i < 32 ? m0 : m1) >> (i & 31)) & 1u)) x[i] = 0.f;
+}
 
 // Packs 64 fp32 values (pairs 2i, 2i+1) into 32 bf16x2 words.
 __device__ __forceinline__ void pack64(const float (&x)[64], uint32_t (&w)[32]) {
@@ -519,13 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
     if (MODE == kDq) {
       const uint32_t tS[2] = {tmem + lane_off + col, tmem + lane_off + 128 + col};
       const uint32_t tDP = tmem + lane_off + 256 + col;
-      float lse2 = 0.f, dsum = 0.f;
+      uint64_t nl2 = 0, nd2 = 0;  // this row's -L log2 e and -D, paired for packed arithmetic
       if (n_cols > 0) {
         ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.row_full, 0));
         const float4 rec = reinterpret_cast<const float4 *>(smem + kSmemRec)[row];
-        lse2 = rec.x;
-        dsum = rec.y;
+        nl2 = ptx::f2_pack(rec.x, rec.x);
+        nd2 = ptx::f2_pack(rec.y, rec.y);
       }
+      const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
       KeyIter it;
       key_first(P, c, it);
       for (int j = 0; ok && j < n_cols; ++j) {
@@ -540,11 +548,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         if (!P.all_full) key_mask(P, c, it, m);
         const uint32_t m0 = m[2 * g], m1 = m[2 * g + 1];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const bool valid = ((i < 32 ? m0 : m1) >> (i & 31)) & 1u;
-          const float p = ptx::ex2(fmaf(s[i], sl2, -lse2));
-          s[i] = valid ? p * (dp[i] - dsum) : 0.f;
+        for (int i = 0; i < 64; i += 2) {
+          float x0, x1, d0, d1;
+          ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(s[i], s[i + 1]), sl2x2, nl2), x0, x1);
+          const uint64_t pp = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
+          ptx::f2_unpack(ptx::fmul2(pp, ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), nd2)), d0, d1);
+          s[i] = d0;
+          s[i + 1] = d1;
         }
+        if ((m0 & m1) != 0xFFFFFFFFu) zero_masked(s, m0, m1);  // warp-uniform: a partial key tile
         uint32_t pk[32];
         pack64(s, pk);
         ptx::tmem_st32(tS[j & 1], pk);  // dS (bf16) over the first half of this thread's S columns
@@ -586,12 +598,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
           m0 = qt.mask[2 * g];
           m1 = qt.mask[2 * g + 1];
         }
+        const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const bool valid = ((i < 32 ? m0 : m1) >> (i & 31)) & 1u;
-          const float e = ptx::ex2(fmaf(p[i], sl2, -rec[i].x));
-          p[i] = valid ? e : 0.f;
+        for (int i = 0; i < 64; i += 2) {
+          float x0, x1;
+          ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(p[i], p[i + 1]), sl2x2, ptx::f2_pack(rec[i].x, rec[i + 1].x)), x0, x1);
+          p[i] = ptx::ex2(x0);
+          p[i + 1] = ptx::ex2(x1);
         }
+        const bool partial = (m0 & m1) != 0xFFFFFFFFu;  // warp-uniform: a partial query tile
+        if (partial) zero_masked(p, m0, m1);
         uint32_t pk[32];
         pack64(p, pk);
         ptx::tmem_st32(tS, pk);  // P^T (bf16) over the first half of this thread's S^T columns
@@ -604,10 +620,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         float dp[64];
         tmem_ld64f(tDP, dp);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const bool valid = ((i < 32 ? m0 : m1) >> (i & 31)) & 1u;
-          dp[i] = valid ? p[i] * (dp[i] - rec[i].y) : 0.f;
+        for (int i = 0; i < 64; i += 2) {
+          float d0, d1;
+          ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(p[i], p[i + 1]),
+                                    ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), ptx::f2_pack(rec[i].y, rec[i + 1].y))),
+                         d0, d1);
+          dp[i] = d0;
+          dp[i + 1] = d1;
         }
+        if (partial) zero_masked(dp, m0, m1);  // dS = 0 there whatever dP holds
         pack64(dp, pk);
         ptx::tmem_st32(tDP, pk);  // dS^T (bf16) over the first half of this thread's dP^T columns
         ptx::tmem_st_wait();
@@ -678,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
   }
 }
 
-// Per query token: {L log2(e), dout . out, 0, 0}, two tokens per warp (16 lanes x
+// Per query token: {-L log2(e), -(dout . out), 0, 0}, two tokens per warp (16 lanes x
 // 8 bf16 each), float32 sums in a fixed order.
 __global__ void __launch_bounds__(256) bwd_records_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
                                                           const float *lse, float4 *rec, long long rows) {
@@ -697,7 +718,7 @@ __global__ void __launch_bounds__(256) bwd_records_kernel(const __nv_bfloat16 *o
   }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-  if (r < rows && part == 0) rec[r] = make_float4(lse[r] * 1.4426950408889634f, acc, 0.f, 0.f);
+  if (r < rows && part == 0) rec[r] = make_float4(-lse[r] * 1.4426950408889634f, -acc, 0.f, 0.f);
 }
 
 // Sums the chunks of the long key tiles in order: pooled rows -> dkvp (float32),
