@@ -50,17 +50,28 @@ using namespace sm100;
 enum Mode { kDq = 0, kDkvWindow = 1, kDkvLong = 2 };
 
 constexpr int kThreads = 320;
-constexpr int kSlots = 4;                                   // ring of 32 KB tiles
+constexpr int kMaxSlots = 5;
 constexpr uint32_t kSmemRow = 0;                            // the two row tiles
-constexpr uint32_t kSmemRing = 2 * kTileBytes;
+constexpr uint32_t kSmemRing = 2 * kTileBytes;              // then a ring of 32 KB tiles
 constexpr uint32_t kRecBytes = kTileRows * 16;              // 128 records of 16 bytes
-constexpr uint32_t kSmemRec = kSmemRing + kSlots * kTileBytes;
-constexpr uint32_t kSmemCtrl = kSmemRec + 2 * kRecBytes;
 constexpr uint32_t kCtrlBytes = 1024;
-constexpr uint32_t kSmemList = kSmemCtrl + kCtrlBytes;
 constexpr int kMaxList = 4096;                              // windows whose query tiles one key tile sees
-constexpr uint32_t kSmemBytes = kSmemList + kMaxList * 2 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
+
+// Shared memory of each pass. dq: row tiles q, dout; five ring slots (three key
+// tiles, two value tiles); each thread reads its own row's record from global
+// memory. dK/dV: row tiles k, v; four slots (query and dout tiles in turn); two
+// record buffers for the streamed query tiles; the window pass adds the list of
+// windows that see its key tile.
+template <int MODE>
+struct Smem {
+  static constexpr int slots = MODE == kDq ? 5 : 4;
+  static constexpr uint32_t rec = kSmemRing + slots * kTileBytes;
+  static constexpr uint32_t ctrl = rec + (MODE == kDq ? 0u : 2 * kRecBytes);
+  static constexpr uint32_t list = ctrl + kCtrlBytes;
+  static constexpr uint32_t bytes = list + (MODE == kDkvWindow ? kMaxList * 2 : 0) + 1024;  // + alignment slack
+  static_assert(bytes <= 227u * 1024u, "shared memory of a pass above the 227 KB a CTA may hold");
+};
 
 struct alignas(64) BwdParams {
   CUtensorMap map_q[kMaxShapes], map_k[kMaxShapes], map_v[kMaxShapes], map_do[kMaxShapes];
@@ -70,6 +81,7 @@ struct alignas(64) BwdParams {
   WindowPlan plan;
   const int32_t *route;
   int32_t *dev_err;
+  const float4 *rec;  // the records, [bh][N] (dq pass: each thread reads its row's)
   const float *dkvp;  // final pooled-key gradients: dkp [bh][Np][128], then dvp
   float *part;        // long key tiles: [bh][tile][chunk][dK | dV][128][128] partial sums
   Geo g;
@@ -86,8 +98,8 @@ struct alignas(64) BwdParams {
 static_assert(sizeof(BwdParams) <= 32764, "window plan too large for the kernel parameter space");
 
 struct Ctrl {
-  uint64_t full[kSlots], empty[kSlots];
-  uint64_t row_full, s_full[2], dp_full, p_full, ds_full, acc_full, drain;
+  uint64_t full[kMaxSlots], empty[kMaxSlots];
+  uint64_t row_full, s_full[2], dp_full, dp_free, p_full, ds_full, acc_full, drain;
   uint32_t tmem_base;
   int abort;
   int n_cols;   // column tiles streamed by this CTA
@@ -176,10 +188,11 @@ __device__ __forceinline__ const PlanTile &q_tile(const BwdParams &P, const QIte
 }
 
 // dq pass ring: key tile j in slot j % 3 (read by S(j) and, much later, dq(j)),
-// value tile j in slot 3 (read by dP(j) only), so the next key tiles load while
-// earlier ones still wait for their dq product.
-__device__ __forceinline__ int dq_slot(int j, bool is_v) { return is_v ? 3 : j % 3; }
-__device__ __forceinline__ uint32_t dq_phase(int j, bool is_v) { return is_v ? (j & 1) : ((j / 3) & 1); }
+// value tile j in slot 3 + j % 2 (read by dP(j) only), so the next key tiles load
+// while earlier ones still wait for their dq product, and value tile j + 1 loads
+// while dP(j) is computed and read.
+__device__ __forceinline__ int dq_slot(int j, bool is_v) { return is_v ? 3 + (j & 1) : j % 3; }
+__device__ __forceinline__ uint32_t dq_phase(int j, bool is_v) { return is_v ? ((j >> 1) & 1) : ((j / 3) & 1); }
 
 // Sets the columns whose mask bit is clear to 0 (m0: columns 0-31, m1: 32-63).
 __device__ __forceinline__ void zero_masked(float (&x)[64], uint32_t m0, uint32_t m1) {
@@ -219,8 +232,10 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid_constant__ BwdParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctrl &c = *reinterpret_cast<Ctrl *>(smem + kSmemCtrl);
-  int16_t *list = reinterpret_cast<int16_t *>(smem + kSmemList);
+  using L = Smem<MODE>;
+  constexpr int kSlots = L::slots;
+  Ctrl &c = *reinterpret_cast<Ctrl *>(smem + L::ctrl);
+  int16_t *list = reinterpret_cast<int16_t *>(smem + L::list);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   // ----------------------------------------------------------- unit of this CTA
@@ -248,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
     ptx::mbar_init(&c.s_full[0], 1);
     ptx::mbar_init(&c.s_full[1], 1);
     ptx::mbar_init(&c.dp_full, 1);
+    ptx::mbar_init(&c.dp_free, 256);
     ptx::mbar_init(&c.p_full, 256);
     ptx::mbar_init(&c.ds_full, 256);
     ptx::mbar_init(&c.acc_full, 1);
@@ -310,9 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
     // are 0, and the MMAs multiply them by 0): tiles when the plan has such rows,
     // and always the record buffers.
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    const uint32_t first = P.plan.zero_fill ? kSmemRow : kSmemRec;
+    const uint32_t first = P.plan.zero_fill ? kSmemRow : L::rec;
     uint4 *z = reinterpret_cast<uint4 *>(smem + first);
-    for (uint32_t i = threadIdx.x; i < (kSmemRec + 2 * kRecBytes - first) / 16; i += kThreads) z[i] = zero;
+    for (uint32_t i = threadIdx.x; i < (L::ctrl - first) / 16; i += kThreads) z[i] = zero;
     ptx::fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -334,11 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       Waiter drain{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
       // row tiles: dq pass q, dout (+ records); dK/dV passes k, v
       if (MODE == kDq) {
-        const uint32_t vr = row_tile.valid_rows;
-        ptx::mbar_arrive_expect_tx(&c.row_full, vr * 512u + vr * 16u);
+        ptx::mbar_arrive_expect_tx(&c.row_full, uint32_t(row_tile.valid_rows) * 512u);
         load_window_tile(P.plan, P.g, P.map_q, row_tile, row_org, bh, row0, &c.row_full);
         load_window_tile(P.plan, P.g, P.map_do, row_tile, row_org, bh, row1, &c.row_full);
-        load_window_records(P.plan, P.g, P.map_rec, row_tile, row_org, bh, smem + kSmemRec, &c.row_full);
       } else if (MODE == kDkvWindow) {
         ptx::mbar_arrive_expect_tx(&c.row_full, uint32_t(row_tile.valid_rows) * 512u);
         load_window_tile(P.plan, P.g, P.map_k, row_tile, row_org, bh, row0, &c.row_full);
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
             if (kv == 0) {  // q tile and its records (record buffer j & 1, freed with the q slot)
               ptx::mbar_arrive_expect_tx(&c.full[slot], uint32_t(tile.valid_rows) * (256u + 16u));
               load_window_tile(P.plan, P.g, P.map_q, tile, it.org, bh, dst, &c.full[slot]);
-              load_window_records(P.plan, P.g, P.map_rec, tile, it.org, bh, smem + kSmemRec + (j & 1) * kRecBytes,
+              load_window_records(P.plan, P.g, P.map_rec, tile, it.org, bh, smem + L::rec + (j & 1) * kRecBytes,
                                   &c.full[slot]);
             } else {
               ptx::mbar_arrive_expect_tx(&c.full[slot], uint32_t(tile.valid_rows) * 256u);
@@ -402,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       drain.wait(&c.row_full, 0);
       if (MODE == kDq) {
         for (int j = max(0, last_k - 2); j <= last_k; ++j) drain.wait(&c.full[dq_slot(j, false)], dq_phase(j, false));
-        if (last_v >= 0) drain.wait(&c.full[dq_slot(last_v, true)], dq_phase(last_v, true));
+        for (int j = max(0, last_v - 1); j <= last_v; ++j) drain.wait(&c.full[dq_slot(j, true)], dq_phase(j, true));
       }
       for (int item = max(0, last - (kSlots - 1)); item <= last; ++item)
         drain.wait(&c.full[item % kSlots], (item / kSlots) & 1);
@@ -424,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         auto kdesc = [&](int j) { return ringK + uint32_t(dq_slot(j, false)) * kTileDesc; };
         auto wait_k = [&](int j) { return wt.wait(&c.full[dq_slot(j, false)], dq_phase(j, false)); };
         auto wait_v = [&](int j) { return wt.wait(&c.full[dq_slot(j, true)], dq_phase(j, true)); };
-        const uint32_t vdesc = ringK + 3u * kTileDesc;
+        auto vdesc = [&](int j) { return ringK + uint32_t(dq_slot(j, true)) * kTileDesc; };
         ok = wait_k(0);
         if (ok) {
           ptx::tc_fence_after();
@@ -434,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         }
         if (ok) {
           ptx::tc_fence_after();
-          issue_ss(tDP, r1, vdesc);  // dP(0) = dout V0^T
+          issue_ss(tDP, r1, vdesc(0));  // dP(0) = dout V0^T
           ptx::mma_commit(&c.dp_full);
-          ptx::mma_commit(&c.empty[3]);
+          ptx::mma_commit(&c.empty[dq_slot(0, true)]);
         }
         if (ok && n_cols > 1) {
           ok = wait_k(1);
@@ -454,15 +468,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
             issue_ss(tS[(j + 1) & 1], r0, kdesc(j + 1));
             ptx::mma_commit(&c.s_full[(j + 1) & 1]);
           }
+          if (j + 1 < n_cols) {
+            // dP(j+1) as soon as every thread holds dP(j) in registers: it runs while
+            // dS(j) is computed, off the chain dS(j) -> dP(j+1) -> dS(j+1)
+            if (!wt.wait(&c.dp_free, j & 1) || !wait_v(j + 1)) break;
+            ptx::tc_fence_after();
+            issue_ss(tDP, r1, vdesc(j + 1));
+            ptx::mma_commit(&c.dp_full);
+            ptx::mma_commit(&c.empty[dq_slot(j + 1, true)]);
+          }
           if (!wt.wait(&c.ds_full, j & 1)) break;
           ptx::tc_fence_after();
-          if (j + 1 < n_cols) {
-            if (!wait_v(j + 1)) break;
-            ptx::tc_fence_after();
-            issue_ss(tDP, r1, vdesc);  // dP(j+1): dP(j) has been read
-            ptx::mma_commit(&c.dp_full);
-            ptx::mma_commit(&c.empty[3]);
-          }
           issue_ts_split(tDQ, tS[j & 1], ringMn + uint32_t(dq_slot(j, false)) * kTileDesc, j > 0);  // dq += dS(j) K_j
           ptx::mma_commit(&c.empty[dq_slot(j, false)]);
         }
@@ -527,9 +543,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       const uint32_t tS[2] = {tmem + lane_off + col, tmem + lane_off + 128 + col};
       const uint32_t tDP = tmem + lane_off + 256 + col;
       uint64_t nl2 = 0, nd2 = 0;  // this row's -L log2 e and -D, paired for packed arithmetic
-      if (n_cols > 0) {
-        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.row_full, 0));
-        const float4 rec = reinterpret_cast<const float4 *>(smem + kSmemRec)[row];
+      int t, y, x;                // (a padding row keeps 0, 0: its dS is 0 as its dout row is 0)
+      if (n_cols > 0 && tile_row_token(P.plan, P.g, row_tile, row_org, row, &t, &y, &x)) {
+        const float4 rec = P.rec[(long long)bh * P.g.N + ((long long)t * P.g.H + y) * P.g.W + x];
         nl2 = ptx::f2_pack(rec.x, rec.x);
         nd2 = ptx::f2_pack(rec.y, rec.y);
       }
@@ -544,6 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         float s[64], dp[64];
         tmem_ld64f(tS[j & 1], s);
         tmem_ld64f(tDP, dp);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&c.dp_free);  // dP(j) is in registers: the MMA may overwrite it
         uint32_t m[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
         if (!P.all_full) key_mask(P, c, it, m);
         const uint32_t m0 = m[2 * g], m1 = m[2 * g + 1];
@@ -591,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tc_fence_after();
         float p[64];
         tmem_ld64f(tS, p);
-        const float4 *rec = reinterpret_cast<const float4 *>(smem + kSmemRec + (j & 1) * kRecBytes) + col;
+        const float4 *rec = reinterpret_cast<const float4 *>(smem + L::rec + (j & 1) * kRecBytes) + col;
         uint32_t m0 = 0xFFFFFFFFu, m1 = 0xFFFFFFFFu;
         if (!P.all_full) {
           const PlanTile &qt = q_tile(P, it);
@@ -806,10 +824,10 @@ template <int MODE>
 basa_status run_bwd(const BwdParams &P, long long blocks, cudaStream_t s) {
   if (blocks <= 0) return BASA_OK;
   if (blocks >= (1ll << 31)) return BASA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(attn_bwd_bf16_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+  if (cudaFuncSetAttribute(attn_bwd_bf16_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<MODE>::bytes) !=
       cudaSuccess)
     return BASA_ERR_CUDA;
-  attn_bwd_bf16_kernel<MODE><<<unsigned(blocks), kThreads, kSmemBytes, s>>>(P);
+  attn_bwd_bf16_kernel<MODE><<<unsigned(blocks), kThreads, Smem<MODE>::bytes, s>>>(P);
   return cudaGetLastError() == cudaSuccess ? BASA_OK : BASA_ERR_CUDA;
 }
 
@@ -838,6 +856,7 @@ basa_status launch_attn_bwd_bf16(const void *q, const void *k, const void *v, co
   P.part = reinterpret_cast<float *>(ws + L.rec);
   float *dkvp = reinterpret_cast<float *>(ws + L.rec + L.part);
   P.dkvp = dkvp;
+  P.rec = rec;
   for (int i = 0; i < P.plan.n_shapes; ++i) {
     const PlanShape &sh = P.plan.shape[i];
     if (!encode_grid_map(&P.map_q[i], q, p, N, sh) || !encode_grid_map(&P.map_k[i], k, p, kv_rows, sh) ||
