@@ -58,16 +58,20 @@ constexpr uint32_t kCtrlBytes = 1024;
 constexpr int kMaxList = 4096;                              // windows whose query tiles one key tile sees
 constexpr uint32_t kTmemCols = 512;
 
+constexpr uint32_t kColRecBytes = 8 * 128 * 4;             // per compute warp: 64 x {-L log2 e}, 64 x {-D}
+
 // Shared memory of each pass. dq: row tiles q, dout; five ring slots (three key
 // tiles, two value tiles); each thread reads its own row's record from global
 // memory. dK/dV: row tiles k, v; four slots (query and dout tiles in turn); two
-// record buffers for the streamed query tiles; the window pass adds the list of
-// windows that see its key tile.
+// record buffers for the streamed query tiles, and per compute warp its 64
+// columns' records as two arrays; the window pass adds the list of windows that
+// see its key tile.
 template <int MODE>
 struct Smem {
   static constexpr int slots = MODE == kDq ? 5 : 4;
   static constexpr uint32_t rec = kSmemRing + slots * kTileBytes;
-  static constexpr uint32_t ctrl = rec + (MODE == kDq ? 0u : 2 * kRecBytes);
+  static constexpr uint32_t col_rec = rec + (MODE == kDq ? 0u : 2 * kRecBytes);
+  static constexpr uint32_t ctrl = col_rec + (MODE == kDq ? 0u : kColRecBytes);
   static constexpr uint32_t list = ctrl + kCtrlBytes;
   static constexpr uint32_t bytes = list + (MODE == kDkvWindow ? kMaxList * 2 : 0) + 1024;  // + alignment slack
   static_assert(bytes <= 227u * 1024u, "shared memory of a pass above the 227 KB a CTA may hold");
@@ -601,6 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       }
     } else {
       const uint32_t tS = tmem + lane_off + col, tDP = tmem + lane_off + 128 + col;
+      float *wrec = reinterpret_cast<float *>(smem + L::col_rec) + (warp - 2) * 128;  // [-L log2 e x 64 | -D x 64]
+      const float4 *nl4 = reinterpret_cast<const float4 *>(wrec), *nd4 = reinterpret_cast<const float4 *>(wrec + 64);
       QIter it;
       if (n_cols > 0) q_first(P, list, MODE, MODE == kDkvLong ? chunk * P.chunk_tiles : 0, it);
       for (int j = 0; ok && j < n_cols; ++j) {
@@ -609,7 +615,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tc_fence_after();
         float p[64];
         tmem_ld64f(tS, p);
-        const float4 *rec = reinterpret_cast<const float4 *>(smem + L::rec + (j & 1) * kRecBytes) + col;
+        {
+          // This warp's 64 query records {-L log2 e, -D, 0, 0}, one load per lane
+          // for two columns, rewritten as two arrays that the loops below read four
+          // values at a time.
+          const float4 *r = reinterpret_cast<const float4 *>(smem + L::rec + (j & 1) * kRecBytes) + col;
+          const float4 a = r[lane], b = r[32 + lane];
+          __syncwarp();  // every lane has read the previous tile's arrays
+          wrec[lane] = a.x;
+          wrec[32 + lane] = b.x;
+          wrec[64 + lane] = a.y;
+          wrec[96 + lane] = b.y;
+          __syncwarp();
+        }
         uint32_t m0 = 0xFFFFFFFFu, m1 = 0xFFFFFFFFu;
         if (!P.all_full) {
           const PlanTile &qt = q_tile(P, it);
@@ -618,11 +636,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         }
         const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          float x0, x1;
-          ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(p[i], p[i + 1]), sl2x2, ptx::f2_pack(rec[i].x, rec[i + 1].x)), x0, x1);
+        for (int i = 0; i < 64; i += 4) {
+          const float4 nl = nl4[i / 4];
+          float x0, x1, x2, x3;
+          ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(p[i], p[i + 1]), sl2x2, ptx::f2_pack(nl.x, nl.y)), x0, x1);
+          ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(p[i + 2], p[i + 3]), sl2x2, ptx::f2_pack(nl.z, nl.w)), x2, x3);
           p[i] = ptx::ex2(x0);
           p[i + 1] = ptx::ex2(x1);
+          p[i + 2] = ptx::ex2(x2);
+          p[i + 3] = ptx::ex2(x3);
         }
         const bool partial = (m0 & m1) != 0xFFFFFFFFu;  // warp-uniform: a partial query tile
         if (partial) zero_masked(p, m0, m1);
@@ -638,13 +660,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         float dp[64];
         tmem_ld64f(tDP, dp);
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          float d0, d1;
+        for (int i = 0; i < 64; i += 4) {
+          const float4 nd = nd4[i / 4];
+          float d0, d1, d2, d3;
           ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(p[i], p[i + 1]),
-                                    ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), ptx::f2_pack(rec[i].y, rec[i + 1].y))),
+                                    ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), ptx::f2_pack(nd.x, nd.y))),
                          d0, d1);
+          ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(p[i + 2], p[i + 3]),
+                                    ptx::fadd2(ptx::f2_pack(dp[i + 2], dp[i + 3]), ptx::f2_pack(nd.z, nd.w))),
+                         d2, d3);
           dp[i] = d0;
           dp[i + 1] = d1;
+          dp[i + 2] = d2;
+          dp[i + 3] = d3;
         }
         if (partial) zero_masked(dp, m0, m1);  // dS = 0 there whatever dP holds
         pack64(dp, pk);
