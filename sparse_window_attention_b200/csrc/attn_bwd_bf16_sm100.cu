@@ -103,7 +103,9 @@ static_assert(sizeof(BwdParams) <= 32764, "window plan too large for the kernel 
 
 struct Ctrl {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
-  uint64_t row_full, s_full[2], dp_full, dp_free, p_full, ds_full, acc_full, drain;
+  // dq pass: s_full[j & 1], dp_full[0], dp_free, ds_full[0]; dK/dV passes: s_full[0],
+  // dp_full[0], and per compute group p_full[g], ds_full[g]
+  uint64_t row_full, s_full[2], dp_full[2], dp_free, p_full[2], ds_full[2], acc_full, drain;
   uint32_t tmem_base;
   int abort;
   int n_cols;   // column tiles streamed by this CTA
@@ -264,12 +266,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       ptx::mbar_init(&c.empty[i], 1);
     }
     ptx::mbar_init(&c.row_full, 1);
-    ptx::mbar_init(&c.s_full[0], 1);
-    ptx::mbar_init(&c.s_full[1], 1);
-    ptx::mbar_init(&c.dp_full, 1);
+    const uint32_t per_group = MODE == kDq ? 256 : 128;  // compute threads that arrive
+    for (int g = 0; g < 2; ++g) {
+      ptx::mbar_init(&c.s_full[g], 1);
+      ptx::mbar_init(&c.dp_full[g], 1);
+      ptx::mbar_init(&c.p_full[g], 128);
+      ptx::mbar_init(&c.ds_full[g], per_group);
+    }
     ptx::mbar_init(&c.dp_free, 256);
-    ptx::mbar_init(&c.p_full, 256);
-    ptx::mbar_init(&c.ds_full, 256);
     ptx::mbar_init(&c.acc_full, 1);
     ptx::mbar_init(&c.drain, 1);
     c.abort = 0;
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         if (ok) {
           ptx::tc_fence_after();
           issue_ss(tDP, r1, vdesc(0));  // dP(0) = dout V0^T
-          ptx::mma_commit(&c.dp_full);
+          ptx::mma_commit(&c.dp_full[0]);
           ptx::mma_commit(&c.empty[dq_slot(0, true)]);
         }
         if (ok && n_cols > 1) {
@@ -478,16 +482,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
             if (!wt.wait(&c.dp_free, j & 1) || !wait_v(j + 1)) break;
             ptx::tc_fence_after();
             issue_ss(tDP, r1, vdesc(j + 1));
-            ptx::mma_commit(&c.dp_full);
+            ptx::mma_commit(&c.dp_full[0]);
             ptx::mma_commit(&c.empty[dq_slot(j + 1, true)]);
           }
-          if (!wt.wait(&c.ds_full, j & 1)) break;
+          if (!wt.wait(&c.ds_full[0], j & 1)) break;
           ptx::tc_fence_after();
           issue_ts_split(tDQ, tS[j & 1], ringMn + uint32_t(dq_slot(j, false)) * kTileDesc, j > 0);  // dq += dS(j) K_j
           ptx::mma_commit(&c.empty[dq_slot(j, false)]);
         }
       } else if (MODE != kDq && ok && n_cols > 0) {
-        // TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384
+        // TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384. Compute group g owns query
+        // columns [64 g, 64 g + 64) of S^T and dP^T; the dV and dK products are issued
+        // per group (the K-steps over its queries) as soon as that group's P^T or dS^T
+        // is in TMEM. S^T and dP^T stay whole N = 128 products (an N = 64 half reads
+        // the same A operand from shared memory for half the work).
         const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
         ok = wt.wait(&c.full[0], 0);
         if (ok) {
@@ -499,31 +507,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         if (ok) {
           ptx::tc_fence_after();
           issue_ss(tDP, r1, ringK + slot_of(1));  // dP^T(0) = V dout0^T
-          ptx::mma_commit(&c.dp_full);
+          ptx::mma_commit(&c.dp_full[0]);
         }
         for (int j = 0; ok && j < n_cols; ++j) {
-          const int qi = 2 * j, di = 2 * j + 1;
-          if (!wt.wait(&c.p_full, j & 1)) break;
-          ptx::tc_fence_after();
-          issue_ts_split(tDV, tS, ringMn + slot_of(di), j > 0);  // dV += P^T(j) dout_j
+          const int qi = 2 * j, di = 2 * j + 1, qn = qi + 2, dn = di + 2;
+          const bool more = j + 1 < n_cols;
+          for (int g = 0; ok && g < 2; ++g) {
+            ok = wt.wait(&c.p_full[g], j & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_ts_group(tDV, tS, ringMn + slot_of(di), g, j > 0 || g > 0);  // dV += P^T(j) dout_j
+          }
+          if (!ok) break;
           ptx::mma_commit(&c.empty[di % kSlots]);
-          if (j + 1 < n_cols) {
-            const int qn = qi + 2;
+          if (more) {
             if (!wt.wait(&c.full[qn % kSlots], (qn / kSlots) & 1)) break;
             ptx::tc_fence_after();
             issue_ss(tS, r0, ringK + slot_of(qn));  // S^T(j+1): P^T(j) has been read by dV
             ptx::mma_commit(&c.s_full[0]);
           }
-          if (!wt.wait(&c.ds_full, j & 1)) break;
-          ptx::tc_fence_after();
-          issue_ts_split(tDK, tDP, ringMn + slot_of(qi), j > 0);  // dK += dS^T(j) q_j
+          for (int g = 0; ok && g < 2; ++g) {
+            ok = wt.wait(&c.ds_full[g], j & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_ts_group(tDK, tDP, ringMn + slot_of(qi), g, j > 0 || g > 0);  // dK += dS^T(j) q_j
+          }
+          if (!ok) break;
           ptx::mma_commit(&c.empty[qi % kSlots]);
-          if (j + 1 < n_cols) {
-            const int dn = di + 2;
+          if (more) {
             if (!wt.wait(&c.full[dn % kSlots], (dn / kSlots) & 1)) break;
             ptx::tc_fence_after();
             issue_ss(tDP, r1, ringK + slot_of(dn));  // dP^T(j+1)
-            ptx::mma_commit(&c.dp_full);
+            ptx::mma_commit(&c.dp_full[0]);
           }
         }
       }
@@ -558,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       key_first(P, c, it);
       for (int j = 0; ok && j < n_cols; ++j) {
         ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.s_full[j & 1], (j >> 1) & 1));
-        if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full, j & 1));
+        if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full[0], j & 1));
         if (!ok) break;
         ptx::tc_fence_after();
         float s[64], dp[64];
@@ -584,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tmem_st32(tS[j & 1], pk);  // dS (bf16) over the first half of this thread's S columns
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&c.ds_full);
+        ptx::mbar_arrive(&c.ds_full[0]);
         key_next(P, c, it);
       }
       if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.acc_full, 0));
@@ -653,8 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tmem_st32(tS, pk);  // P^T (bf16) over the first half of this thread's S^T columns
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&c.p_full);
-        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full, j & 1));
+        ptx::mbar_arrive(&c.p_full[g]);
+        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full[0], j & 1));
         if (!ok) break;
         ptx::tc_fence_after();
         float dp[64];
@@ -679,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tmem_st32(tDP, pk);  // dS^T (bf16) over the first half of this thread's dP^T columns
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&c.ds_full);
+        ptx::mbar_arrive(&c.ds_full[g]);
         q_next(P, list, MODE, n_windows, it);
       }
       if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.acc_full, 0));

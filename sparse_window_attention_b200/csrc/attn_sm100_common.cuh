@@ -79,6 +79,18 @@ __device__ __forceinline__ void issue_ts_split(uint32_t d_tmem, uint32_t a_tmem,
                       kIdescBMnMajor, (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// The K-steps of issue_ts_split that read group g's half: K rows [64 g, 64 g + 64)
+// of B and A columns [a + 64 g, a + 64 g + 32).
+__device__ __forceinline__ void issue_ts_group(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, int g,
+                                               bool accumulate) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int kk = 4 * g + i;
+    ptx::mma_bf16_ts2(d_tmem, a_tmem + 64 * g + i * 8, b_lo + ((kk * 2048) >> 4), kDescHi, kIdescBMnMajor,
+                      (accumulate || i > 0) ? 1u : 0u);
+  }
+}
+
 __device__ __forceinline__ int wrap(int x, int g) { return x >= g ? x - g : x; }
 
 // Issue the TMA loads of one 128-row tile of a window (query, key or value tile):
