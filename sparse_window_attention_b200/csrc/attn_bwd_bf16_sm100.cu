@@ -103,9 +103,9 @@ static_assert(sizeof(BwdParams) <= 32764, "window plan too large for the kernel 
 
 struct Ctrl {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
-  // dq pass: s_full[j & 1], dp_full[0], dp_free, ds_full[0]; dK/dV passes: s_full[0],
+  // dq pass: a_ready, s_full[0], s_free, dp_full[0], ds_full[0]; dK/dV passes: s_full[0],
   // dp_full[0], and per compute group p_full[g], ds_full[g]
-  uint64_t row_full, s_full[2], dp_full[2], dp_free, p_full[2], ds_full[2], acc_full, drain;
+  uint64_t row_full, s_full[2], dp_full[2], s_free, a_ready, p_full[2], ds_full[2], acc_full, drain;
   uint32_t tmem_base;
   int abort;
   int n_cols;   // column tiles streamed by this CTA
@@ -234,6 +234,21 @@ __device__ __forceinline__ void stage_row_half(uint8_t *tile, int row, int half,
                       ptx::pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
 }
 
+// Reads 64 bf16 values (columns [64 half, 64 half + 64) of row `row`) from a swizzled
+// 128-row tile as 32 bf16x2 words, the layout of an MMA A operand in TMEM.
+__device__ __forceinline__ void load_row_half(const uint8_t *tile, int row, int half, uint32_t (&w)[32]) {
+  const uint8_t *base = tile + uint32_t(half) * kHalfBytes + uint32_t(row) * 128u;
+  const uint32_t swz = row & 7;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(base + ((uint32_t(c) ^ swz) << 4));
+    w[4 * c] = v.x;
+    w[4 * c + 1] = v.y;
+    w[4 * c + 2] = v.z;
+    w[4 * c + 3] = v.w;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid_constant__ BwdParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -273,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       ptx::mbar_init(&c.p_full[g], 128);
       ptx::mbar_init(&c.ds_full[g], per_group);
     }
-    ptx::mbar_init(&c.dp_free, 256);
+    ptx::mbar_init(&c.s_free, 256);
+    ptx::mbar_init(&c.a_ready, 256);
     ptx::mbar_init(&c.acc_full, 1);
     ptx::mbar_init(&c.drain, 1);
     c.abort = 0;
@@ -441,54 +457,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       auto slot_of = [](int item) { return uint32_t(item % kSlots) * kTileDesc; };
       bool ok = n_cols == 0 || wt.wait(&c.row_full, 0);
       if (MODE == kDq && ok && n_cols > 0) {
-        // TMEM: S buffers at 0 and 128, dP at 256, dq at 384
-        const uint32_t tS[2] = {tmem, tmem + 128}, tDP = tmem + 256, tDQ = tmem + 384;
+        // TMEM: S at 0; dP at 128, with dS written over its first halves; dq at 256; the
+        // q and dout row tiles at 384 and 448 (bf16), copied there once by the compute
+        // warps, so S and dP read their A operand from TMEM and only the key or value
+        // tile from shared memory. Order per key tile j: S(j+1) once every thread holds
+        // S(j) in registers (it runs while P(j) is computed), then dq(j) += dS(j) K_j,
+        // then dP(j+1) over dS(j).
+        const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256, tQ = tmem + 384, tDO = tmem + 448;
         auto kdesc = [&](int j) { return ringK + uint32_t(dq_slot(j, false)) * kTileDesc; };
         auto wait_k = [&](int j) { return wt.wait(&c.full[dq_slot(j, false)], dq_phase(j, false)); };
         auto wait_v = [&](int j) { return wt.wait(&c.full[dq_slot(j, true)], dq_phase(j, true)); };
         auto vdesc = [&](int j) { return ringK + uint32_t(dq_slot(j, true)) * kTileDesc; };
-        ok = wait_k(0);
+        ok = wt.wait(&c.a_ready, 0) && wait_k(0);
         if (ok) {
           ptx::tc_fence_after();
-          issue_ss(tS[0], r0, kdesc(0));  // S(0) = q K0^T
+          issue_ts_kmajor(tS, tQ, kdesc(0));  // S(0) = q K0^T
           ptx::mma_commit(&c.s_full[0]);
           ok = wait_v(0);
         }
         if (ok) {
           ptx::tc_fence_after();
-          issue_ss(tDP, r1, vdesc(0));  // dP(0) = dout V0^T
+          issue_ts_kmajor(tDP, tDO, vdesc(0));  // dP(0) = dout V0^T
           ptx::mma_commit(&c.dp_full[0]);
           ptx::mma_commit(&c.empty[dq_slot(0, true)]);
         }
-        if (ok && n_cols > 1) {
-          ok = wait_k(1);
-          if (ok) {
-            ptx::tc_fence_after();
-            issue_ss(tS[1], r0, kdesc(1));  // S(1)
-            ptx::mma_commit(&c.s_full[1]);
-          }
-        }
         for (int j = 0; ok && j < n_cols; ++j) {
-          if (j >= 1 && j + 1 < n_cols) {
-            // S(j+1) into the buffer dq(j-1) has finished reading
-            if (!wait_k(j + 1)) break;
+          const bool more = j + 1 < n_cols;
+          if (more) {
+            if (!wt.wait(&c.s_free, j & 1) || !wait_k(j + 1)) break;
             ptx::tc_fence_after();
-            issue_ss(tS[(j + 1) & 1], r0, kdesc(j + 1));
-            ptx::mma_commit(&c.s_full[(j + 1) & 1]);
-          }
-          if (j + 1 < n_cols) {
-            // dP(j+1) as soon as every thread holds dP(j) in registers: it runs while
-            // dS(j) is computed, off the chain dS(j) -> dP(j+1) -> dS(j+1)
-            if (!wt.wait(&c.dp_free, j & 1) || !wait_v(j + 1)) break;
-            ptx::tc_fence_after();
-            issue_ss(tDP, r1, vdesc(j + 1));
-            ptx::mma_commit(&c.dp_full[0]);
-            ptx::mma_commit(&c.empty[dq_slot(j + 1, true)]);
+            issue_ts_kmajor(tS, tQ, kdesc(j + 1));  // S(j+1)
+            ptx::mma_commit(&c.s_full[0]);
           }
           if (!wt.wait(&c.ds_full[0], j & 1)) break;
           ptx::tc_fence_after();
-          issue_ts_split(tDQ, tS[j & 1], ringMn + uint32_t(dq_slot(j, false)) * kTileDesc, j > 0);  // dq += dS(j) K_j
+          issue_ts_split(tDQ, tDP, ringMn + uint32_t(dq_slot(j, false)) * kTileDesc, j > 0);  // dq += dS(j) K_j
           ptx::mma_commit(&c.empty[dq_slot(j, false)]);
+          if (more) {
+            if (!wait_v(j + 1)) break;
+            ptx::tc_fence_after();
+            issue_ts_kmajor(tDP, tDO, vdesc(j + 1));  // dP(j+1), after dq(j) has read dS(j)
+            ptx::mma_commit(&c.dp_full[0]);
+            ptx::mma_commit(&c.empty[dq_slot(j + 1, true)]);
+          }
         }
       } else if (MODE != kDq && ok && n_cols > 0) {
         // TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384. Compute group g owns query
@@ -559,8 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
     const float sl2 = P.scale_log2;
     bool ok = true;
     if (MODE == kDq) {
-      const uint32_t tS[2] = {tmem + lane_off + col, tmem + lane_off + 128 + col};
-      const uint32_t tDP = tmem + lane_off + 256 + col;
+      const uint32_t tS = tmem + lane_off + col, tDP = tmem + lane_off + 128 + col;
       uint64_t nl2 = 0, nd2 = 0;  // this row's -L log2 e and -D, paired for packed arithmetic
       int t, y, x;                // (a padding row keeps 0, 0: its dS is 0 as its dout row is 0)
       if (n_cols > 0 && tile_row_token(P.plan, P.g, row_tile, row_org, row, &t, &y, &x)) {
@@ -568,35 +578,58 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         nl2 = ptx::f2_pack(rec.x, rec.x);
         nd2 = ptx::f2_pack(rec.y, rec.y);
       }
+      if (n_cols > 0) {
+        // This row's q and dout (this group's 64 of the head dims) into TMEM, where the
+        // MMAs read them as the A operand of S and dP.
+        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.row_full, 0));
+        if (ok) {
+          uint32_t w[32];
+          load_row_half(row0, row, g, w);
+          ptx::tmem_st32(tmem + lane_off + 384 + 32 * g, w);
+          load_row_half(row1, row, g, w);
+          ptx::tmem_st32(tmem + lane_off + 448 + 32 * g, w);
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&c.a_ready);
+        }
+      }
       const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
       KeyIter it;
       key_first(P, c, it);
       for (int j = 0; ok && j < n_cols; ++j) {
-        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.s_full[j & 1], (j >> 1) & 1));
-        if (ok) ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full[0], j & 1));
+        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.s_full[0], j & 1));
         if (!ok) break;
         ptx::tc_fence_after();
         float s[64], dp[64];
-        tmem_ld64f(tS[j & 1], s);
-        tmem_ld64f(tDP, dp);
+        tmem_ld64f(tS, s);
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&c.dp_free);  // dP(j) is in registers: the MMA may overwrite it
+        ptx::mbar_arrive(&c.s_free);  // S(j) is in registers: the MMA may overwrite it
         uint32_t m[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
         if (!P.all_full) key_mask(P, c, it, m);
         const uint32_t m0 = m[2 * g], m1 = m[2 * g + 1];
 #pragma unroll
         for (int i = 0; i < 64; i += 2) {
-          float x0, x1, d0, d1;
+          float x0, x1;
           ptx::f2_unpack(ptx::ffma2(ptx::f2_pack(s[i], s[i + 1]), sl2x2, nl2), x0, x1);
-          const uint64_t pp = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
-          ptx::f2_unpack(ptx::fmul2(pp, ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), nd2)), d0, d1);
+          s[i] = ptx::ex2(x0);
+          s[i + 1] = ptx::ex2(x1);
+        }
+        ok = __all_sync(0xFFFFFFFFu, wt.wait(&c.dp_full[0], j & 1));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        tmem_ld64f(tDP, dp);
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          float d0, d1;
+          ptx::f2_unpack(ptx::fmul2(ptx::f2_pack(s[i], s[i + 1]), ptx::fadd2(ptx::f2_pack(dp[i], dp[i + 1]), nd2)), d0,
+                         d1);
           s[i] = d0;
           s[i + 1] = d1;
         }
         if ((m0 & m1) != 0xFFFFFFFFu) zero_masked(s, m0, m1);  // warp-uniform: a partial key tile
         uint32_t pk[32];
         pack64(s, pk);
-        ptx::tmem_st32(tS[j & 1], pk);  // dS (bf16) over the first half of this thread's S columns
+        ptx::tmem_st32(tDP, pk);  // dS (bf16) over the first half of this thread's dP columns
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&c.ds_full[0]);
@@ -606,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       if (ok) {
         ptx::tc_fence_after();
         float x[64];
-        tmem_ld64f(tmem + lane_off + 384 + col, x);
+        tmem_ld64f(tmem + lane_off + 256 + col, x);
 #pragma unroll
         for (int i = 0; i < 64; ++i) x[i] *= P.scale;
         stage_row_half(row0, row, g, x);  // the q tile is no longer read

@@ -79,6 +79,16 @@ __device__ __forceinline__ void issue_ts_split(uint32_t d_tmem, uint32_t a_tmem,
                       kIdescBMnMajor, (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// D (=) A B^T over head_dim 128 with A (bf16, 128 rows x 128) in TMEM, 8 columns per
+// K-step of 16, and B a token-major tile in shared memory read K-major as in issue_ss.
+__device__ __forceinline__ void issue_ts_kmajor(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    ptx::mma_bf16_ts2(d_tmem, a_tmem + kk * 8, b_lo + off, kDescHi, kIdescKMajor, kk > 0 ? 1u : 0u);
+  }
+}
+
 // The K-steps of issue_ts_split that read group g's half: K rows [64 g, 64 g + 64)
 // of B and A columns [a + 64 g, a + 64 g + 32).
 __device__ __forceinline__ void issue_ts_group(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, int g,
