@@ -14,8 +14,9 @@
 //   records      per query token {-L log2(e), -D} (16-byte records, TMA-loadable with
 //                the same boxes as the query tiles; negated for the packed FMA/add)
 //   dq pass      one CTA per (b*head, window, query tile): the key stream of the
-//                forward; S = q K^T and dP = dout V^T on tcgen05 (two S buffers in
-//                TMEM), dS by the compute warps, dq += dS K accumulated in TMEM.
+//                forward; q and dout copied once into TMEM, so S = q K^T and
+//                dP = dout V^T read their A operand from TMEM; dS by the compute
+//                warps (written over dP), dq += dS K accumulated in TMEM.
 //   dK/dV long   (pooled and text key tiles, which every query of the head sees)
 //                one CTA per (b*head, key tile, chunk of the head's query tiles):
 //                S^T = K q^T, dP^T = V dout^T, dV += P^T dout, dK += dS^T q in TMEM;
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
     if (lane == 0) {
       Waiter wt{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, true};
       Waiter drain{&c.abort, P.dev_err, P.timeout_ns, BASA_DEVERR_TIMEOUT_PRODUCER, false};
-      // row tiles: dq pass q, dout (+ records); dK/dV passes k, v
+      // row tiles: dq pass q, dout; dK/dV passes k, v
       if (MODE == kDq) {
         ptx::mbar_arrive_expect_tx(&c.row_full, uint32_t(row_tile.valid_rows) * 512u);
         load_window_tile(P.plan, P.g, P.map_q, row_tile, row_org, bh, row0, &c.row_full);
