@@ -95,6 +95,7 @@ struct alignas(64) BwdParams {
   float inv_patch;
   float scale_log2;  // log2(e) / sqrt(d)
   float scale;       // 1 / sqrt(d)
+  uint32_t flags;    // basa_params.flags (test hook: skip the first ring load)
   int all_full;      // every tile of the streams is full: no column masks
   int max_tiles;     // most tiles of a window type
   int n_chunks, chunk_tiles, q_tiles;  // long mode: query tiles of a head, split in chunks
@@ -393,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
         ptx::tma_load_3d(row1 + kHalfBytes, mv, &c.row_full, 64, row, bh);
       }
       int last = -1, last_k = -1, last_v = -1;
+      bool skipped0 = false;  // test hook: the first ring item was never loaded
       if (MODE == kDq) {
         KeyIter it;
         key_first(P, c, it);
@@ -401,6 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = dq_slot(j, kv == 1);
             if (!wt.wait(&c.empty[slot], dq_phase(j, kv == 1) ^ 1)) { ok = false; break; }
+            if (j == 0 && kv == 0 && (P.flags & BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD)) {
+              skipped0 = true;
+              last_k = 0;
+              continue;
+            }
             const uint32_t bytes = it.seg <= P.routed_k
                                        ? uint32_t(P.plan.tile[P.plan.type[c.wtype[it.seg]].first_tile + it.t].valid_rows) * 256u
                                        : kTileBytes;
@@ -420,6 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
           for (int kv = 0; kv < 2; ++kv) {
             const int item = 2 * j + kv, slot = item % kSlots;
             if (!wt.wait(&c.empty[slot], ((item / kSlots) & 1) ^ 1)) { ok = false; break; }
+            if (item == 0 && (P.flags & BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD)) {
+              skipped0 = true;
+              last = 0;
+              continue;
+            }
             uint8_t *dst = smem + kSmemRing + slot * kTileBytes;
             if (kv == 0) {  // q tile and its records (record buffer j & 1, freed with the q slot)
               ptx::mbar_arrive_expect_tx(&c.full[slot], uint32_t(tile.valid_rows) * (256u + 16u));
@@ -440,11 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_bf16_kernel(const __grid
       // A slot's earlier copies completed before the slot was granted again.
       drain.wait(&c.row_full, 0);
       if (MODE == kDq) {
-        for (int j = max(0, last_k - 2); j <= last_k; ++j) drain.wait(&c.full[dq_slot(j, false)], dq_phase(j, false));
+        for (int j = max(0, last_k - 2); j <= last_k; ++j)
+          if (j > 0 || !skipped0) drain.wait(&c.full[dq_slot(j, false)], dq_phase(j, false));
         for (int j = max(0, last_v - 1); j <= last_v; ++j) drain.wait(&c.full[dq_slot(j, true)], dq_phase(j, true));
       }
       for (int item = max(0, last - (kSlots - 1)); item <= last; ++item)
-        drain.wait(&c.full[item % kSlots], (item / kSlots) & 1);
+        if (item > 0 || !skipped0) drain.wait(&c.full[item % kSlots], (item / kSlots) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -969,6 +982,7 @@ basa_status launch_attn_bwd_bf16(const void *q, const void *k, const void *v, co
   P.chunk_tiles = L.chunk_tiles;
   P.q_tiles = L.q_tiles;
   P.timeout_ns = (p.wait_timeout_us ? (unsigned long long)p.wait_timeout_us : 2000000ull) * 1000ull;
+  P.flags = p.flags;
 
   const long long rows = bh * N;
   bwd_records_kernel<<<unsigned((rows + 15) / 16), 256, 0, s>>>(

@@ -136,17 +136,19 @@ class BasaLayer:
             ws = self.text_workspace
         B.basa_text_attn_fwd(q_text, k, v, out_text, ws, self.params((0, 0, 0)), stream)
 
-    def backward(self, q, k, v, out, lse, dout, shift, stream=None):
+    def backward(self, q, k, v, out, lse, dout, shift, stream=None, **extra):
         """dq, dk, dv of the attention (basa_window_attn_bwd: bfloat16 on the tensor
         cores, or float32) for the pooled K/V and routed windows currently held by
-        the layer; `lse` is the forward's log-sum-exp over all keys."""
+        the layer; `lse` is the forward's log-sum-exp over all keys. ``extra`` goes
+        into the parameters (e.g. ``wait_timeout_us``, ``flags``)."""
         dq = torch.empty_like(q)
         dk = torch.empty_like(k)
         dv = torch.empty_like(v)
-        nbytes = B.basa_window_attn_bwd_workspace_bytes(self.params(shift))
+        params = self.params(shift, **extra)
+        nbytes = B.basa_window_attn_bwd_workspace_bytes(params)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device) if nbytes else None
-        B.basa_window_attn_bwd(q, k, v, self.kp, self.vp, self.route_idx, out, lse, dout, dq, dk, dv, ws,
-                               self.params(shift), stream)
+        B.basa_window_attn_bwd(q, k, v, self.kp, self.vp, self.route_idx, out, lse, dout, dq, dk, dv, ws, params,
+                               stream)
         return dq, dk, dv
 
     def forward(self, q, k, v, shift, out=None, stream=None):
