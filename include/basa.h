@@ -84,8 +84,10 @@ typedef enum { BASA_BF16 = 0, BASA_F32 = 1 } basa_dtype;
 #define BASA_DEVERR_BAD_ROUTE 0x8
 
 /* Test hook for basa_params.flags: the attention kernel's loader skips the TMA
- * load of the first key tile, so every wait on it runs into its time limit and
- * the kernel returns with BASA_DEVERR_TIMEOUT_* set. Never set in normal use. */
+ * load of the first key tile (the bfloat16 backward: each pass skips its first
+ * ring load, a key tile in the dq pass and a query tile in the dK/dV passes), so
+ * every wait on it runs into its time limit and the kernel returns with
+ * BASA_DEVERR_TIMEOUT_* set. Never set in normal use. */
 #define BASA_FLAG_TEST_SKIP_FIRST_KEY_LOAD 0x1u
 
 typedef struct {
