@@ -59,16 +59,6 @@ __device__ __forceinline__ void issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint3
     ptx::mma_bf16_ts2(d_tmem, a_tmem + kk * 8, b_lo + ((kk * 2048) >> 4), kDescHi, kIdescBMnMajor,
                       (accumulate || kk > 0) ? 1u : 0u);
 }
-// One half of issue_ts: K-steps 0-3 (h = 0, A columns [a, a + 32)) or 4-7 (h = 1,
-// columns [a + 32, a + 64)), for an A operand written in two halves.
-__device__ __forceinline__ void issue_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, int h, bool accumulate) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int kk = 4 * h + i;
-    ptx::mma_bf16_ts2(d_tmem, a_tmem + kk * 8, b_lo + ((kk * 2048) >> 4), kDescHi, kIdescBMnMajor,
-                      (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
 // Split layout: K 0-63 at columns [a, a + 32), K 64-127 at [a + 64, a + 96), so two
 // warpgroups that each own 64 columns of a 128-column fp32 buffer can write their
 // packed bf16 halves in place without touching the other's inputs.
