@@ -883,11 +883,13 @@ int head_query_tiles(const basa_params &p, const WindowPlan &plan) {
   return n;
 }
 
-// Chunking of the pooled / text key tiles' query range: enough CTAs for about two
-// waves of a 148-SM part, at least 4 query tiles per chunk. It depends on the shape
-// only, so the workspace size and the order of the chunk sums (hence the bits of the
-// results) are the same on every device.
-constexpr long long kLongTargetCtas = 2 * 148;
+// Chunking of the pooled / text key tiles' query range: the chunk count n (at
+// least 4 query tiles per chunk) that minimises the estimated time of the launch,
+// waves x (tiles per chunk + a CTA's fixed start and end cost in tiles), for a
+// 148-SM part. It depends on the shape only, so the workspace size and the order of
+// the chunk sums (hence the bits of the results) are the same on every device.
+constexpr long long kLongSms = 148;
+constexpr double kLongCtaCostTiles = 3.5;
 BwdLayout bwd_layout(const basa_params &p, const WindowPlan &plan) {
   BwdLayout L{};
   const long long bh = (long long)p.B * p.heads;
@@ -896,12 +898,20 @@ BwdLayout bwd_layout(const basa_params &p, const WindowPlan &plan) {
   L.n_long = (n_pool + kTileRows - 1) / kTileRows + (p.n_text + kTileRows - 1) / kTileRows;
   L.q_tiles = head_query_tiles(p, plan);
   L.n_chunks = 1;
-  if (L.n_long > 0) {
+  L.chunk_tiles = L.q_tiles;
+  if (L.n_long > 0 && L.q_tiles > 0) {
     const long long units = bh * L.n_long;
-    long long want = (kLongTargetCtas + units - 1) / units;
-    want = std::max(1LL, std::min<long long>(want, std::max(1, L.q_tiles / 4)));
-    L.chunk_tiles = int((L.q_tiles + want - 1) / want);
-    L.n_chunks = (L.q_tiles + L.chunk_tiles - 1) / L.chunk_tiles;
+    double best = -1.0;
+    for (int n = 1; n <= std::max(1, L.q_tiles / 4); ++n) {
+      const int tiles = (L.q_tiles + n - 1) / n;
+      const int chunks = (L.q_tiles + tiles - 1) / tiles;
+      const double cost = double((units * chunks + kLongSms - 1) / kLongSms) * (tiles + kLongCtaCostTiles);
+      if (best < 0.0 || cost < best) {
+        best = cost;
+        L.chunk_tiles = tiles;
+        L.n_chunks = chunks;
+      }
+    }
   }
   L.rec = align256(size_t(bh) * N * 16);
   L.part = align256(size_t(bh) * L.n_long * L.n_chunks * 2 * kTileRows * 128 * sizeof(float));
