@@ -201,3 +201,33 @@ def test_route_workspace_bytes():
     p = _p(routed_k=2)
     assert B.basa_route_workspace_bytes(p) == 2 * 1 * 2 * 16 * 128 * 4
     assert B.basa_route_workspace_bytes(_p(head_dim=100)) == 0
+
+
+def _bwd_chunks(wl, shift):
+    """Chunk count of the bfloat16 backward's pooled/text key pass, read back from
+    the workspace size (records + chunk partials + pooled-key gradients)."""
+    p = B.make_params(wl.B, wl.heads, wl.d, wl.grid, wl.window, shift, wl.pool, wl.n_text, wl.routed_k, wl.dtype,
+                      route_radius=wl.route_radius)
+    bh = wl.B * wl.heads
+    n = wl.grid[0] * wl.grid[1] * wl.grid[2]
+    pt, ph, pw = wl.pool
+    n_pool = (wl.grid[0] // pt) * (wl.grid[1] // ph) * (wl.grid[2] // pw)
+    n_long = -(-n_pool // 128) + -(-wl.n_text // 128)
+    up = lambda x: (x + 255) // 256 * 256
+    part = B.basa_window_attn_bwd_workspace_bytes(p) - up(bh * n * 16) - up(bh * n_pool * 128 * 4 * 2)
+    assert part % (bh * n_long * 2 * 128 * 128 * 4) == 0
+    return part // (bh * n_long * 2 * 128 * 128 * 4), bh * n_long
+
+
+def test_backward_chunking_fills_whole_waves():
+    """The pooled/text pass splits each head's query tiles into the chunk count that
+    minimises waves x (tiles per chunk + a CTA's fixed cost) on 148 SMs: one chunk
+    (144 CTAs, one wave) at FLUX 2048^2 and 1024^2, six on Wan (144 CTAs), where
+    the earlier rule of about two waves gave 2.9 and 2.1 waves."""
+    from sparse_window_attention_b200 import synth
+
+    for name, want in (("flux2k", 1), ("flux1k", 1), ("wan", 6)):
+        wl = synth.WORKLOADS[name]
+        chunks, units = _bwd_chunks(wl, synth.SHIFT_CYCLES[name][-1])
+        assert chunks == want, (name, chunks)
+        assert units * chunks <= 148, (name, units * chunks)  # one wave
