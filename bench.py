@@ -87,9 +87,10 @@ bus = sys.argv[1]
 h = pynvml.nvmlDeviceGetHandleByPciBusId(bus) if bus else pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
 print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
 while True:
-    t = time.time()
-    print(f"{t:.6f} {pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)} "
-          f"{int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))}", flush=True)
+    ta = time.time()
+    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+    print(f"{ta:.6f} {time.time():.6f} {mhz} {bits}", flush=True)
     time.sleep(0.0005)
 """
 
@@ -143,6 +144,10 @@ class ClockSampler:
         if self.proc is not None:
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # let the poll loop reach its steady rate before the timed region starts
+            deadline = time.time() + 2.0
+            while len(self.lines) < 2 and time.time() < deadline:
+                time.sleep(0.001)
         return self
 
     def _read(self):
@@ -170,11 +175,14 @@ class ClockSampler:
         nvml = self.source is not None and self.source.startswith("nvml")
         for line in self.lines:
             if nvml:
+                # "t mhz bits", or "ta tb mhz bits": a query made over [ta, tb]; kept
+                # when it overlaps the timed region
                 parts = line.split()
-                if len(parts) != 3:
+                if len(parts) not in (3, 4):
                     continue
-                t, mhz, bits = float(parts[0]), float(parts[1]), int(parts[2])
-                if self.t0 is not None and not (self.t0 <= t <= self.t1):
+                ta, tb = float(parts[0]), float(parts[-3])
+                mhz, bits = float(parts[-2]), int(parts[-1])
+                if self.t0 is not None and (tb < self.t0 or ta > self.t1):
                     continue
                 sm.append(mhz)
                 reasons.update(n for n, b in self.REASONS if bits & b)

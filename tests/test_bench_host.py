@@ -31,6 +31,10 @@ def test_clock_samples_outside_the_timed_region_are_dropped():
     out = s.summary()
     assert out["samples"] == 2 and out["sm_mhz"] == (1965 + 1900) / 2
     assert out["reasons"] == ["sw_power_cap"]  # hw_slowdown and hw_thermal_slowdown fell outside
+    # interval samples ("ta tb mhz bits"): a query that overlaps the region counts
+    s.lines = ["99.990 100.0007 1700 0", "100.0026 100.004 1800 0", "100.0010 100.0012 1965 0"]
+    out = s.summary()
+    assert out["samples"] == 2 and out["sm_mhz"] == (1700 + 1965) / 2
 
 
 def test_reference_arm_prints_one_contract_line(repo_root):
